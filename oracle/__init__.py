@@ -1,0 +1,24 @@
+"""CPU float64 oracle for the paged KV pool hot path.
+
+TEST INFRASTRUCTURE ONLY: imported by ``tests/``, ``__graft_entry__.smoke()``
+and the CPU-baseline leg of ``bench.py``; never by the library.  It shares no
+code with the CUDA path.
+
+Parity status per function (what pins it, in ``tests/test_oracle_pins.py``):
+  store_kv, slots_of, gather_kv -- closed forms (bit copy; hand-derived page
+      translation fixture in tests/golden) and brute force;
+  attend, decode_attn, extend_attn -- brute-force dense attention on tiny
+      inputs, a two-key closed form, and the invariants (slot permutation,
+      chunked == unchunked, shared prefix == private copy, one-token context
+      returns V, constant K returns mean V, decode == extend with one row,
+      q*c with k/c, identical query heads);
+  partial_state, combine_states -- merging split states equals the unsplit
+      result.
+The pages print no worked numerical example for any of these, so no stored
+value comes from them.
+"""
+from .paged_attention import (attend, combine_states, decode_attn, extend_attn, gather_kv,
+                              partial_state, slots_of, store_kv, to_f64)
+
+__all__ = ["attend", "combine_states", "decode_attn", "extend_attn", "gather_kv",
+           "partial_state", "slots_of", "store_kv", "to_f64"]
