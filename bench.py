@@ -1,0 +1,537 @@
+"""Benchmark of the paged KV pool hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload decode-qwen3-0.6b|decode-qwen3-8b|chunked-prefill|radix-prefix]
+
+Default workload (one "step"): the Qwen3-0.6B-shaped decode step -- 64
+requests with contexts uniform in [512, 4096], Hq 16, Hkv 8, d 128, bf16,
+page_size 1 over a 300k-slot, 28-layer pool (layer 13): store_kv of the 64
+new tokens, then decode_attn (split-KV partials + combine).  The metric is
+decode KV GB/s: K/V bytes of every context token (all KV heads, both planes)
+plus page-table, query and output bytes, divided by device time.  Inputs are
+larger than L2 (~0.6 GB of KV per step), so no L2 flush is needed.
+
+Under torchrun each rank runs an independent replica on its own GPU (the
+path needs no collective); value = total bytes of all ranks / max-over-ranks
+time, "scaling": "weak".
+
+``--impl reference`` times the float64 CPU oracle on a bounded sample of the
+same workload and prints the same JSON line with "impl": "reference".
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+HBM_FALLBACK_GBS = 6650.0
+BF16_FALLBACK_TFLOPS = 1590.0
+
+
+# ---------------------------------------------------------------------------
+# helpers
+# ---------------------------------------------------------------------------
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), "measured"
+    except Exception:
+        return HBM_FALLBACK_GBS, BF16_FALLBACK_TFLOPS, 1400.0, "fallback"
+
+
+def source_hash(*names):
+    h = hashlib.sha256()
+    for n in names:
+        with open(os.path.join(ROOT, "paged_kv_gqa_scatter_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str, src_hash: str):
+    """Per-launch DRAM bytes of `kernel` from the committed ncu summary, or None
+    when the kernel's source has changed since the counters were taken."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        e = d.get(kernel)
+        if e and e.get("source_hash") == src_hash:
+            return float(e["dram_bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup():
+    import torch
+    import torch.distributed as dist
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        n = [i.get("num_threads", 1) for i in info if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+# ---------------------------------------------------------------------------
+# decode workload (the headline)
+# ---------------------------------------------------------------------------
+def decode_bytes(wl) -> int:
+    """Algorithmic bytes of one decode_attn call: every context token's K and V
+    rows (all KV heads), its page-table entry (one per token at page_size 1, one
+    per page otherwise), the queries and the outputs."""
+    B, Hq = wl.batch, wl.num_q_heads
+    esz = 2 if wl.pool.dtype == "bf16" else 4
+    n = wl.seq_lens.astype(np.int64)
+    row = wl.pool.num_kv_heads * 128 * esz
+    P = wl.pool.page_size
+    table = int(n.sum()) * 4 if P == 1 else int(((n + P - 1) // P).sum()) * 4
+    return int(n.sum()) * 2 * row + table + 2 * B * Hq * 128 * esz + 8 * B
+
+
+def store_bytes(wl) -> int:
+    esz = 2 if wl.pool.dtype == "bf16" else 4
+    row = wl.pool.num_kv_heads * 128 * esz
+    return wl.batch * (4 * row + 4)
+
+
+def cpu_decode_sample(wl, budget_s: float = 12.0):
+    """Time the oracle on the first requests of the workload until ~budget_s of
+    CPU work; return (GB/s in the metric's bytes, sample description)."""
+    import oracle
+    from paged_kv_gqa_scatter_b200 import workloads as W
+    kp = {l: a for l, a in wl.k_planes.items()} if isinstance(wl.k_planes, dict) else wl.k_planes
+    vp = {l: a for l, a in wl.v_planes.items()} if isinstance(wl.v_planes, dict) else wl.v_planes
+    done, nbytes = 0, 0
+    esz = 2 if wl.pool.dtype == "bf16" else 4
+    row = wl.pool.num_kv_heads * 128 * esz
+    t0 = time.perf_counter()
+    for r in range(wl.batch):
+        oracle.decode_attn(wl.q, kp, vp, wl.layer, wl.page_table, wl.table_idx, wl.seq_lens,
+                           wl.pool.page_size, wl.scale, requests=[r])
+        n = int(wl.seq_lens[r])
+        nbytes += n * (2 * row + 4) + 2 * wl.num_q_heads * 128 * esz + 8
+        done += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return nbytes / dt / 1e9, f"oracle decode_attn on the first {done} of {wl.batch} requests " \
+                              f"({nbytes / 1e6:.1f} MB of KV), float64 numpy", dt
+
+
+def run_decode(args, world, rank, local):
+    import torch
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    from paged_kv_gqa_scatter_b200 import api, _lib
+    from paged_kv_gqa_scatter_b200 import workloads as W
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if args.workload == "decode-qwen3-8b":
+        free, _ = torch.cuda.mem_get_info()
+        bytes_per_page = 36 * 16 * 8 * 128 * 2 * 2
+        num_pages = int(0.6 * free // bytes_per_page)
+        wl = W.decode_qwen3_8b(num_pages=num_pages)
+        layers = list(range(wl.pool.num_layers))
+    else:
+        wl = W.decode_qwen3_06b()
+        layers = [wl.layer]
+    lib = _lib.load()
+
+    # ---- device residency (inputs resident in HBM before the timed region) ----
+    def tdev(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    spec = wl.pool
+    pool = api.KVPool.empty(spec.num_layers, spec.num_slots, spec.num_kv_heads, page_size=spec.page_size,
+                            device=dev, zero=not isinstance(wl.k_planes, W.TiledPlane))
+    if isinstance(wl.k_planes, W.TiledPlane):
+        for plane, dst in ((wl.k_planes, pool.k), (wl.v_planes, pool.v)):
+            blk = tdev(plane.block)
+            flat = dst.view(-1, spec.num_kv_heads, 128)
+            nb = blk.shape[0]
+            for s in range(0, flat.shape[0], nb):
+                m = min(nb, flat.shape[0] - s)
+                flat[s:s + m].copy_(blk[:m])
+    else:
+        for l in layers:
+            pool.k[l].copy_(tdev(wl.k_planes[l]))
+            pool.v[l].copy_(tdev(wl.v_planes[l]))
+    table = api.PageTable(torch.from_numpy(wl.page_table).to(dev))
+    table_idx = torch.from_numpy(wl.table_idx).to(dev)
+    seq_lens = torch.from_numpy(wl.seq_lens).to(dev)
+    q = tdev(wl.q)
+    k_new = tdev(wl.k_new)
+    v_new = tdev(wl.v_new)
+    out_loc = torch.from_numpy(wl.out_loc).to(dev)
+    out = torch.empty_like(q)
+    ws = api.decode_workspace(wl.batch, wl.num_q_heads, device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        for l in layers:
+            api.store_kv(pool, l, k_new, v_new, out_loc, err)
+            api.decode_attn(pool, l, q, table, table_idx, seq_lens, out, ws, scale=wl.scale, dev_err=err)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    # ---- timed region: K steps, events per call on the launching stream ------
+    nL = len(layers)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps * nL)]
+    start = torch.cuda.Event(enable_timing=True)
+    stop = torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks.start()
+    start.record(stream)
+    i = 0
+    for _ in range(args.steps):
+        for l in layers:
+            ev[i][0].record(stream)
+            api.store_kv(pool, l, k_new, v_new, out_loc, err)
+            ev[i][1].record(stream)
+            api.decode_attn(pool, l, q, table, table_idx, seq_lens, out, ws, scale=wl.scale, dev_err=err)
+            ev[i][2].record(stream)
+            i += 1
+    stop.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    ms_total = start.elapsed_time(stop)
+    ms_total = max_over_ranks(ms_total, world)
+    dec_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    st_ms = [e[0].elapsed_time(e[1]) for e in ev]
+    errv = int(err.item())
+
+    per_call = decode_bytes(wl)
+    step_bytes = nL * (per_call + store_bytes(wl))
+    value = world * step_bytes * args.steps / (ms_total / 1e3) / 1e9
+    hbm, bf16, bf16s, peak_src = measured_peaks()
+    dec_avg_ms = sum(dec_ms) / len(dec_ms)
+    achieved = per_call / (dec_avg_ms / 1e3) / 1e9
+    traffic = recorded_traffic("decode_split_kernel", source_hash("decode.cu", "common.cuh"))
+
+    # ---- e2e through the C ABI with host buffers -------------------------------
+    import torch as _t
+    h_q = _t.from_numpy(np.ascontiguousarray(wl.q).view(np.int16)).pin_memory()
+    h_k = _t.from_numpy(np.ascontiguousarray(wl.k_new).view(np.int16)).pin_memory()
+    h_v = _t.from_numpy(np.ascontiguousarray(wl.v_new).view(np.int16)).pin_memory()
+    h_loc = _t.from_numpy(wl.out_loc).pin_memory()
+    h_sl = _t.from_numpy(wl.seq_lens).pin_memory()
+    h_ti = _t.from_numpy(wl.table_idx).pin_memory()
+    h_pt = _t.from_numpy(wl.page_table).pin_memory()
+    h_out = _t.empty(out.shape, dtype=_t.int16).pin_memory()
+    h2d = sum(x.numel() * x.element_size() for x in (h_q, h_k, h_v, h_loc, h_sl, h_ti, h_pt))
+    d2h = h_out.numel() * h_out.element_size()
+
+    def e2e_step():
+        q.view(_t.int16).copy_(h_q, non_blocking=True)
+        k_new.view(_t.int16).copy_(h_k, non_blocking=True)
+        v_new.view(_t.int16).copy_(h_v, non_blocking=True)
+        out_loc.copy_(h_loc, non_blocking=True)
+        seq_lens.copy_(h_sl, non_blocking=True)
+        table_idx.copy_(h_ti, non_blocking=True)
+        table.entries.copy_(h_pt, non_blocking=True)
+        for l in layers:
+            api.store_kv(pool, l, k_new, v_new, out_loc, err)
+            api.decode_attn(pool, l, q, table, table_idx, seq_lens, out, ws, scale=wl.scale, dev_err=err)
+        h_out.copy_(out.view(_t.int16), non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+    e2e_val = world * step_bytes * args.steps / (e2e_ms / 1e3) / 1e9
+
+    result = {
+        "metric": "paged decode-attn KV GB/s",
+        "value": round(value, 2),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_total / args.steps, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded PCG64 N(0,1) values rounded to bf16; K x0.5)" if wl.name.endswith("0.6b")
+                else "synthetic (seeded PCG64 N(0,1) block tiled over the pool)",
+        "config": {
+            "workload": wl.name,
+            "batch": wl.batch,
+            "context_tokens": int(wl.seq_lens.sum()),
+            "num_q_heads": wl.num_q_heads, "num_kv_heads": spec.num_kv_heads, "head_dim": 128,
+            "page_size": spec.page_size, "pool_slots": spec.num_slots, "pool_layers": spec.num_layers,
+            "layers_per_step": nL,
+            "step": "store_kv + decode_attn (split partials + combine) per layer",
+            "l2": "inputs larger than L2 (no flush)",
+            "parallelism": f"replicas x{world}",
+        },
+        "decode_tok_per_s_per_layer": round(world * wl.batch * args.steps * nL / (ms_total / 1e3) / nL, 1),
+        "decode_call_us": round(dec_avg_ms * 1e3, 2),
+        "store_kv_call_us": round(sum(st_ms) / len(st_ms) * 1e3, 2),
+        "roofline": {
+            "kernel": "decode_attn (decode_split_kernel + decode_combine_kernel, timed together)",
+            "bound": "hbm",
+            "achieved": round(achieved, 1),
+            "peak": hbm,
+            "peak_source": peak_src,
+            "unit": "GB/s",
+            "frac": round(achieved / hbm, 4),
+            "traffic": traffic,
+            "algorithmic_bytes_per_launch": per_call,
+        },
+        "e2e": {"value": round(e2e_val, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": 3 * args.steps * nL,
+        "device_error_word": errv,
+        "clocks": clk,
+    }
+    if args.workload == "decode-qwen3-8b":
+        result["config"]["alias_factor"] = round(getattr(wl, "alias_factor", 0.0), 3)
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        gbs, sample, _ = cpu_decode_sample(wl)
+        result["cpu_baseline"] = {"value": round(gbs, 4), "unit": "GB/s", "cores": blas_threads(),
+                                  "kind": "oracle", "sample": sample}
+    if not args.no_extend and args.workload == "decode-qwen3-0.6b":
+        result["extend"] = run_extend_measure(dev, warmup=3, iters=max(5, args.steps))
+    return result
+
+
+def run_extend_measure(dev, warmup=3, iters=10):
+    """Extend TFLOP/s on the chunked-prefill step (2048-token chunk at prefix 6144,
+    Hq 32, Hkv 8): causal FLOPs = 4 d Hq (e p + e (e+1) / 2)."""
+    import torch
+    from paged_kv_gqa_scatter_b200 import api
+    from paged_kv_gqa_scatter_b200 import workloads as W
+    mix = W.chunked_prefill_step(step=3)
+    wl = mix.extend
+
+    def tdev(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    spec = wl.pool
+    pool = api.KVPool.empty(spec.num_layers, spec.num_slots, spec.num_kv_heads, device=dev)
+    pool.k[0].copy_(tdev(wl.k_planes[0]))
+    pool.v[0].copy_(tdev(wl.v_planes[0]))
+    table = api.PageTable(torch.from_numpy(wl.page_table).to(dev))
+    ti = torch.from_numpy(wl.table_idx).to(dev)
+    pl = torch.from_numpy(wl.prefix_lens).to(dev)
+    el = torch.from_numpy(wl.extend_lens).to(dev)
+    qo = torch.from_numpy(wl.q_offsets).to(dev)
+    q = tdev(wl.q)
+    out = torch.empty_like(q)
+    api.store_kv(pool, 0, tdev(wl.k_new), tdev(wl.v_new), torch.from_numpy(wl.out_loc).to(dev))
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    mx = int(wl.extend_lens.max())
+    for _ in range(warmup):
+        api.extend_attn(pool, 0, q, table, ti, pl, el, qo, mx, out, scale=wl.scale, dev_err=err)
+    torch.cuda.synchronize()
+    s = torch.cuda.current_stream(dev)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(iters)]
+    for a, b in evs:
+        a.record(s)
+        api.extend_attn(pool, 0, q, table, ti, pl, el, qo, mx, out, scale=wl.scale, dev_err=err)
+        b.record(s)
+    torch.cuda.synchronize()
+    ms = sorted(a.elapsed_time(b) for a, b in evs)
+    med = ms[len(ms) // 2]
+    flops = 4 * 128 * wl.num_q_heads * wl.causal_pairs()
+    _, bf16, _, src = measured_peaks()
+    tf = flops / (med / 1e3) / 1e12
+    return {"workload": "chunked-prefill extend, 2048-token chunk at prefix 6144, Hq 32 Hkv 8",
+            "tflops": round(tf, 2), "ms": round(med, 4), "flops": flops,
+            "roofline": {"bound": "tensor", "achieved": round(tf, 2), "peak": bf16,
+                         "peak_source": src, "unit": "TFLOP/s", "frac": round(tf / bf16, 4)},
+            "device_error_word": int(err.item())}
+
+
+# ---------------------------------------------------------------------------
+# reference arm: the float64 oracle on the host cores
+# ---------------------------------------------------------------------------
+def run_reference(args, world, rank):
+    from paged_kv_gqa_scatter_b200 import workloads as W
+    if rank != 0:
+        return None
+    wl = W.decode_qwen3_06b()
+    budget = float(os.environ.get("PKV_REF_STEP_SECONDS", "4"))
+    for _ in range(args.warmup):
+        cpu_decode_sample(wl, budget_s=0.5)
+    vals, secs, sample = [], 0.0, ""
+    for _ in range(args.steps):
+        v, sample, dt = cpu_decode_sample(wl, budget_s=budget)
+        vals.append(v)
+        secs += dt
+    value = statistics.median(vals)
+    cores = blas_threads()
+    return {
+        "impl": "reference",
+        "metric": "paged decode-attn KV GB/s",
+        "value": round(value, 4),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(secs / args.steps * 1e3, 2),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic (seeded PCG64 N(0,1) values rounded to bf16; K x0.5)",
+        "config": {"workload": wl.name, "batch": wl.batch, "num_q_heads": wl.num_q_heads,
+                   "num_kv_heads": wl.pool.num_kv_heads, "head_dim": 128, "page_size": 1,
+                   "pool_slots": wl.pool.num_slots, "pool_layers": wl.pool.num_layers},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+                         "sample": sample + f"; {budget:.0f} s per step"},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="decode-qwen3-0.6b",
+                    choices=["decode-qwen3-0.6b", "decode-qwen3-8b"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extend", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        res = run_reference(args, world, rank)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return 0
+    world, rank, local = dist_setup()
+    res = run_decode(args, world, rank, local)
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

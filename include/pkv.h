@@ -1,0 +1,237 @@
+/*
+ * pkv.h -- C ABI of the paged KV pool attention library (sm_100a / B200).
+ *
+ * The library implements the GPU hot path of a mini-SGLang-style serving
+ * engine: scattering each step's new K/V rows into a paged pool, and GQA
+ * attention over that pool through a token-granular page table, for decode
+ * (one query token per request) and for extend (a prefill chunk attending
+ * causally to its cached prefix and to itself).
+ *
+ * Sources (web pages on mini-SGLang, cited by title and section):
+ *   [P5] "Mini-SGLang 完整剖析" (blog.rzhang-lab.cn/post/3)
+ *        §1.2 prefill vs decode, §1.3 KV cache, §1.4 paged pool and prefix
+ *        sharing, §4.2.3 request length fields, §4.4.3 pool tensor,
+ *        §4.6.4 page-table metadata, §4.6.7 attention layer / store_kv,
+ *        §4.9.4 store kernel shape checks.
+ *   [P4] "深入解析 mini-sglang" (yunpan.plus), chunked prefill.
+ *   [P3] "mini-sglang 深度分析报告" (nightvoyager.top), design notes
+ *        (page_size-1 page table).
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * Ownership: the caller owns every buffer passed in (device memory unless a
+ *   parameter says "host").  No call keeps a pointer after it returns, and no
+ *   call allocates device memory; scratch space comes from a caller-provided
+ *   workspace whose size a *_workspace_bytes query returns.
+ * Streams: every compute call is asynchronous on the given stream (0 = the
+ *   legacy default stream) and never synchronises the host.
+ * Errors: calls return a pkv_status.  Host-side checks (null pointers,
+ *   negative sizes, unsupported dtype or head_dim, misaligned strides, a
+ *   workspace that is too small) return an error before anything is
+ *   launched.  Data-dependent faults found on the device (a slot or page
+ *   table index out of range, an empty context) are not trapped: the
+ *   offending element is skipped or zero-filled, and a bit from
+ *   pkv_device_error is OR-ed into the caller's `dev_err` word (a device
+ *   int32, may be NULL).  No kernel traps, asserts or waits without bound:
+ *   each internal wait gives up after about one second and sets
+ *   PKV_DEV_ERR_TIMEOUT.
+ * Element types: bf16 (the product path) and fp32 (a check build of the same
+ *   kernels for tighter numerical comparison).  head_dim must be 128.
+ */
+#ifndef PKV_H_
+#define PKV_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef void* pkv_stream_t; /* a cudaStream_t */
+
+typedef enum {
+  PKV_OK = 0,
+  PKV_ERR_INVALID_ARG = 1,      /* null pointer, negative size, bad stride   */
+  PKV_ERR_UNSUPPORTED = 2,      /* dtype, head_dim or head counts not built  */
+  PKV_ERR_MISALIGNED = 3,       /* a pointer or stride breaks 16-byte rules  */
+  PKV_ERR_WORKSPACE = 4,        /* workspace missing or too small            */
+  PKV_ERR_CUDA = 5,             /* a CUDA runtime call failed                */
+  PKV_ERR_TOO_LARGE = 6         /* a size beyond a documented maximum        */
+} pkv_status;
+
+typedef enum {
+  PKV_DEV_ERR_SLOT_RANGE = 1,    /* a slot (out_loc or table entry) >= num_slots or < 0 */
+  PKV_DEV_ERR_TABLE_RANGE = 2,   /* table_idx row or column beyond the table            */
+  PKV_DEV_ERR_EMPTY_CONTEXT = 4, /* decode seq_len < 1, or queries with no key          */
+  PKV_DEV_ERR_BAD_LENGTH = 8,    /* negative prefix/extend length, or q_offsets broken  */
+  PKV_DEV_ERR_PAGE_ALIGN = 16,   /* page_size > 1 and a page's first entry % page_size  */
+  PKV_DEV_ERR_TIMEOUT = 32       /* an internal wait gave up (never expected)           */
+} pkv_device_error;
+
+typedef enum { PKV_DTYPE_BF16 = 0, PKV_DTYPE_F32 = 1 } pkv_dtype;
+
+/*
+ * The KV pool [P5 §4.4.3; §1.4].
+ *
+ * The pages store K and V in one tensor (2, layers, pages, page_size,
+ * kv_heads, head_dim) and address it flattened to slots (pages*page_size,
+ * kv_heads, head_dim).  Here K and V are two planes with the same geometry,
+ * each [num_layers][num_slots][num_kv_heads][head_dim], head_dim contiguous
+ * and kv heads adjacent within a slot; `layer_stride` and `slot_stride` are
+ * element strides between consecutive layers and slots (slot_stride >=
+ * num_kv_heads*head_dim).  Slot s of page p and offset o is s = p*page_size
+ * + o.  `k` and `v` must be 16-byte aligned and slot_stride*element_size a
+ * multiple of 16.  The caller owns the planes.
+ */
+typedef struct {
+  void* k;
+  void* v;
+  int64_t num_layers;
+  int64_t num_slots;
+  int64_t layer_stride;
+  int64_t slot_stride;
+  int32_t num_kv_heads;
+  int32_t head_dim;
+  int32_t page_size;
+  int32_t dtype; /* pkv_dtype */
+} pkv_pool;
+
+/*
+ * The page table [P5 §4.6.4; P3 design notes].
+ *
+ * int32 [rows][cols] with row stride `row_stride` (elements), token
+ * granular: entry [row][j] is the slot of token j of the request that owns
+ * row `row`.  With page_size P > 1 the kernels follow the slice-and-divide
+ * reading of the pages: the page of token j is entry [row][P*(j/P)] / P and
+ * its slot is page*P + j%P (so only each page's first entry is read; it must
+ * be a multiple of P).  `table_idx[r]` (int32, one per request) selects the
+ * row of request r [P5 §6.1 table_idx; P4 chunked prefill: all chunks of a
+ * request share one row].
+ */
+typedef struct {
+  const int32_t* entries;
+  int64_t rows;
+  int64_t cols;
+  int64_t row_stride;
+} pkv_page_table;
+
+/* Returns a static, human-readable string for a pkv_status or device-error bit set. */
+const char* pkv_status_string(int status);
+
+/* Library version string (static). */
+const char* pkv_version(void);
+
+/*
+ * store_kv [P5 §4.6.7: the backend first scatters the step's new K/V into
+ * the pool at batch.out_loc; §4.9.4: k/v are [L, D] with a row stride,
+ * indices are int32 or int64, the pool rows are [-1, D]].
+ *
+ *   pool.k[layer][out_loc[i]][:] = k[i*k_row_stride .. + Hkv*head_dim)
+ *   pool.v[layer][out_loc[i]][:] = v[i*v_row_stride .. + Hkv*head_dim)
+ *   for 0 <= i < n_tokens, as a bit copy in the pool's element type.
+ *
+ * k, v: device, element type = pool.dtype, row strides in elements (k and v
+ *   are typically column slices of a fused qkv output); both pointers and
+ *   strides must keep rows 16-byte aligned.
+ * out_loc: device, int32 (out_loc_is_i64 = 0) or int64 (= 1), n_tokens entries.
+ *   Slots must be distinct within one call (the pages give every new token
+ *   its own slot); an out-of-range slot is skipped and sets
+ *   PKV_DEV_ERR_SLOT_RANGE.
+ * n_tokens == 0 is a no-op.
+ */
+int pkv_store_kv(const pkv_pool* pool, int32_t layer, const void* k, int64_t k_row_stride,
+                 const void* v, int64_t v_row_stride, const void* out_loc,
+                 int32_t out_loc_is_i64, int64_t n_tokens, int32_t* dev_err,
+                 pkv_stream_t stream);
+
+/*
+ * gather_kv -- copies requests' K/V rows, in token order, through the page
+ * table into dense buffers [P5 §4.6.4 page-table translation].  It is the
+ * translation step the attention kernels perform internally, exposed on its
+ * own so that it can be checked bit for bit.
+ *
+ *   k_out[row_offsets[r] + j][:] = pool.k[layer][slot(r, j)][:]  (same for v)
+ *   for 0 <= j < seq_lens[r], 0 <= r < batch.
+ *
+ * table_idx, seq_lens: device int32 [batch]; row_offsets: device int64
+ * [batch+1] (exclusive prefix sum of seq_lens, computed by the caller);
+ * k_out, v_out: device, [row_offsets[batch]][Hkv*head_dim], pool dtype.
+ * A slot out of range zero-fills the row and sets PKV_DEV_ERR_SLOT_RANGE.
+ */
+int pkv_gather_kv(const pkv_pool* pool, int32_t layer, const pkv_page_table* table,
+                  const int32_t* table_idx, const int32_t* seq_lens, const int64_t* row_offsets,
+                  int32_t batch, void* k_out, void* v_out, int32_t* dev_err,
+                  pkv_stream_t stream);
+
+/*
+ * decode_attn [P5 §1.2: decode processes one token per request and is
+ * memory-bandwidth bound; §4.6.4: cache_seqlens is each request's total KV
+ * length; §4.6.7: store_kv runs before the kernel, so the context includes
+ * the token just stored; §4.5.3: KV heads are shared by Hq/Hkv query heads].
+ *
+ *   out[r][h][:] = sum_j softmax_j(scale * q[r][h] . K_r[j][h/G]) V_r[j][h/G]
+ *   over j < seq_lens[r], G = num_q_heads / pool.num_kv_heads,
+ *   K_r[j] = pool.k[layer][slot(r, j)], V_r likewise.
+ *
+ * q: device [batch][num_q_heads][head_dim] contiguous, pool dtype.
+ * out: device [batch][num_q_heads][head_dim] contiguous, pool dtype
+ *   (fp32 accumulation, rounded to nearest-even on store).
+ * table_idx, seq_lens: device int32 [batch].
+ * scale: softmax scale (the pages do not state it; 1/sqrt(head_dim) is the
+ *   usual choice).
+ * workspace: device scratch of at least pkv_decode_workspace_bytes(batch,
+ *   num_q_heads) bytes, 16-byte aligned, owned by the caller, not shared by
+ *   calls that may overlap on the GPU.
+ * Supported: head_dim 128, num_kv_heads 1..8, num_q_heads/num_kv_heads in
+ *   {1, 2, 4, 8}.  seq_lens[r] < 1 writes a zero row and sets
+ *   PKV_DEV_ERR_EMPTY_CONTEXT.  batch == 0 is a no-op.
+ * The work is split across the context (split-KV): one persistent grid
+ * walks (request, chunk) items, then a second kernel merges the chunks of
+ * requests that had more than one.
+ */
+size_t pkv_decode_workspace_bytes(int32_t batch, int32_t num_q_heads);
+int pkv_decode_attn(const pkv_pool* pool, int32_t layer, const void* q, int32_t num_q_heads,
+                    const pkv_page_table* table, const int32_t* table_idx,
+                    const int32_t* seq_lens, int32_t batch, float scale, void* out,
+                    void* workspace, size_t workspace_bytes, int32_t* dev_err,
+                    pkv_stream_t stream);
+
+/*
+ * extend_attn [P4 chunked prefill: every chunk of a request uses the same
+ * table row and reuses the KV of the chunks before it; P5 §4.2.3: a request
+ * has cached_len (its prefix, possibly radix-shared) and extend_len =
+ * device_len - cached_len new tokens; §1.4: requests sharing a prefix point
+ * their table rows at the same slots; §1.2: prefill is compute bound].
+ *
+ *   For request r with p = prefix_lens[r], e = extend_lens[r], query row
+ *   i < e sits at position p + i and attends causally to keys 0 .. p + i:
+ *   out[q_offsets[r] + i][h][:] = sum_{j <= p+i} softmax_j(scale * q[..][h]
+ *   . K_r[j][h/G]) V_r[j][h/G].  The chunk's own K/V must already be in the
+ *   pool (store_kv first, as the pages do).
+ *
+ * q, out: device [total_q][num_q_heads][head_dim] contiguous, pool dtype.
+ * prefix_lens, extend_lens: device int32 [batch]; q_offsets: device int32
+ *   [batch+1], q_offsets[0] = 0, q_offsets[r+1] = q_offsets[r] + extend_lens[r],
+ *   q_offsets[batch] = total_q.
+ * max_extend_len: host int, an upper bound on every extend_lens[r] (used to
+ *   size the launch; rows beyond it are not computed and set
+ *   PKV_DEV_ERR_BAD_LENGTH).
+ * workspace: pkv_extend_workspace_bytes(...) bytes (currently 0 for bf16).
+ * The bf16 path runs QK^T and PV on the tcgen05 tensor cores with TMEM
+ * accumulators; the fp32 check build uses CUDA cores.  Same support limits
+ * as decode_attn.
+ */
+size_t pkv_extend_workspace_bytes(int32_t batch, int32_t num_q_heads, int64_t total_q);
+int pkv_extend_attn(const pkv_pool* pool, int32_t layer, const void* q, int32_t num_q_heads,
+                    const pkv_page_table* table, const int32_t* table_idx,
+                    const int32_t* prefix_lens, const int32_t* extend_lens,
+                    const int32_t* q_offsets, int32_t batch, int64_t total_q,
+                    int32_t max_extend_len, float scale, void* out, void* workspace,
+                    size_t workspace_bytes, int32_t* dev_err, pkv_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PKV_H_ */

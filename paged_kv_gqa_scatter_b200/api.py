@@ -1,0 +1,173 @@
+"""Torch-facing binding of the pkv C ABI: same call names, marshalling only.
+
+PyTorch provides device memory and streams; every step of the path runs in
+the CUDA kernels of ``libpkv.so``.  Each call passes ``tensor.data_ptr()``
+values and the current CUDA stream to the C entry point and raises
+``PkvError`` on a non-zero status.  There is no CPU path.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+from typing import Optional
+
+import torch
+
+from . import _lib
+
+DTYPE_CODES = {torch.bfloat16: 0, torch.float32: 1}
+HEAD_DIM = 128
+
+
+def _stream_ptr(stream: Optional[torch.cuda.Stream]) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return int(s.cuda_stream)
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else int(t.data_ptr())
+
+
+def _require_cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("pkv calls take CUDA tensors")
+
+
+class KVPool:
+    """K and V planes ``[num_layers][num_slots][num_kv_heads][128]`` (caller memory).
+
+    ``k`` and ``v`` may be views with any layer/slot strides as long as each
+    slot's heads and dims are contiguous (the pool layout of include/pkv.h).
+    """
+
+    def __init__(self, k: torch.Tensor, v: torch.Tensor, page_size: int = 1):
+        if k.shape != v.shape or k.dtype != v.dtype or k.dim() != 4:
+            raise ValueError("k and v must be matching 4-D tensors")
+        if k.stride(3) != 1 or k.stride(2) != k.shape[3] or v.stride() != k.stride():
+            raise ValueError("heads and dims of a slot must be contiguous, same strides for k and v")
+        if k.dtype not in DTYPE_CODES:
+            raise ValueError(f"unsupported pool dtype {k.dtype}")
+        _require_cuda(k, v)
+        self.k, self.v = k, v
+        self.page_size = int(page_size)
+        self.c = _lib.PkvPool(
+            k=k.data_ptr(), v=v.data_ptr(), num_layers=k.shape[0], num_slots=k.shape[1],
+            layer_stride=k.stride(0), slot_stride=k.stride(1), num_kv_heads=k.shape[2],
+            head_dim=k.shape[3], page_size=self.page_size, dtype=DTYPE_CODES[k.dtype])
+
+    @classmethod
+    def empty(cls, num_layers, num_slots, num_kv_heads, dtype=torch.bfloat16, page_size=1,
+              device="cuda", zero=True):
+        mk = torch.zeros if zero else torch.empty
+        k = mk((num_layers, num_slots, num_kv_heads, HEAD_DIM), dtype=dtype, device=device)
+        v = mk((num_layers, num_slots, num_kv_heads, HEAD_DIM), dtype=dtype, device=device)
+        return cls(k, v, page_size)
+
+    @property
+    def num_kv_heads(self) -> int:
+        return self.k.shape[2]
+
+    @property
+    def dtype(self):
+        return self.k.dtype
+
+
+class PageTable:
+    """int32 ``[rows][cols]`` token-granular page table (a CUDA tensor view)."""
+
+    def __init__(self, entries: torch.Tensor):
+        if entries.dtype != torch.int32 or entries.dim() != 2 or entries.stride(1) != 1:
+            raise ValueError("page table must be a 2-D int32 tensor with contiguous rows")
+        _require_cuda(entries)
+        self.entries = entries
+        self.c = _lib.PkvPageTable(entries=entries.data_ptr(), rows=entries.shape[0],
+                                   cols=entries.shape[1], row_stride=entries.stride(0))
+
+
+def store_kv(pool: KVPool, layer: int, k: torch.Tensor, v: torch.Tensor, out_loc: torch.Tensor,
+             dev_err: Optional[torch.Tensor] = None, stream=None) -> None:
+    """pkv_store_kv: scatter rows of k/v ([N][Hkv*128], row-strided) to out_loc."""
+    _require_cuda(k, v, out_loc, dev_err)
+    if k.dim() == 3:
+        k = k.reshape(k.shape[0], -1)
+    if v.dim() == 3:
+        v = v.reshape(v.shape[0], -1)
+    if k.stride(1) != 1 or v.stride(1) != 1 or k.dtype != pool.dtype or v.dtype != pool.dtype:
+        raise ValueError("k/v rows must be contiguous and of the pool dtype")
+    if out_loc.dtype not in (torch.int32, torch.int64) or not out_loc.is_contiguous():
+        raise ValueError("out_loc must be contiguous int32 or int64")
+    lib = _lib.load()
+    _lib.check(lib.pkv_store_kv(ctypes.byref(pool.c), layer, k.data_ptr(), k.stride(0),
+                                v.data_ptr(), v.stride(0), out_loc.data_ptr(),
+                                1 if out_loc.dtype == torch.int64 else 0, out_loc.shape[0],
+                                _ptr(dev_err), _stream_ptr(stream)), "store_kv")
+
+
+def gather_kv(pool: KVPool, layer: int, table: PageTable, table_idx: torch.Tensor,
+              seq_lens: torch.Tensor, row_offsets: torch.Tensor, k_out: torch.Tensor,
+              v_out: torch.Tensor, dev_err: Optional[torch.Tensor] = None, stream=None) -> None:
+    """pkv_gather_kv: copy each request's rows through the table into k_out/v_out."""
+    _require_cuda(table_idx, seq_lens, row_offsets, k_out, v_out, dev_err)
+    lib = _lib.load()
+    _lib.check(lib.pkv_gather_kv(ctypes.byref(pool.c), layer, ctypes.byref(table.c),
+                                 table_idx.data_ptr(), seq_lens.data_ptr(), row_offsets.data_ptr(),
+                                 seq_lens.shape[0], k_out.data_ptr(), v_out.data_ptr(),
+                                 _ptr(dev_err), _stream_ptr(stream)), "gather_kv")
+
+
+def decode_workspace_bytes(batch: int, num_q_heads: int) -> int:
+    return int(_lib.load().pkv_decode_workspace_bytes(batch, num_q_heads))
+
+
+def decode_workspace(batch: int, num_q_heads: int, device="cuda") -> torch.Tensor:
+    n = decode_workspace_bytes(batch, num_q_heads)
+    return torch.empty(max(16, n), dtype=torch.uint8, device=device)
+
+
+def decode_attn(pool: KVPool, layer: int, q: torch.Tensor, table: PageTable,
+                table_idx: torch.Tensor, seq_lens: torch.Tensor, out: torch.Tensor,
+                workspace: torch.Tensor, scale: Optional[float] = None,
+                dev_err: Optional[torch.Tensor] = None, stream=None) -> None:
+    """pkv_decode_attn: q [B][Hq][128] -> out [B][Hq][128] over each request's context."""
+    _require_cuda(q, table_idx, seq_lens, out, workspace, dev_err)
+    if not (q.is_contiguous() and out.is_contiguous()):
+        raise ValueError("q and out must be contiguous")
+    if q.dtype != pool.dtype or out.dtype != pool.dtype:
+        raise ValueError("q/out dtype must match the pool")
+    B, Hq, D = q.shape
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    lib = _lib.load()
+    _lib.check(lib.pkv_decode_attn(ctypes.byref(pool.c), layer, q.data_ptr(), Hq,
+                                   ctypes.byref(table.c), table_idx.data_ptr(), seq_lens.data_ptr(),
+                                   B, scale, out.data_ptr(), workspace.data_ptr(),
+                                   workspace.numel() * workspace.element_size(), _ptr(dev_err),
+                                   _stream_ptr(stream)), "decode_attn")
+
+
+def extend_workspace_bytes(batch: int, num_q_heads: int, total_q: int) -> int:
+    return int(_lib.load().pkv_extend_workspace_bytes(batch, num_q_heads, total_q))
+
+
+def extend_attn(pool: KVPool, layer: int, q: torch.Tensor, table: PageTable,
+                table_idx: torch.Tensor, prefix_lens: torch.Tensor, extend_lens: torch.Tensor,
+                q_offsets: torch.Tensor, max_extend_len: int, out: torch.Tensor,
+                scale: Optional[float] = None, workspace: Optional[torch.Tensor] = None,
+                dev_err: Optional[torch.Tensor] = None, stream=None) -> None:
+    """pkv_extend_attn: causal attention of each request's chunk over prefix + chunk."""
+    _require_cuda(q, table_idx, prefix_lens, extend_lens, q_offsets, out, workspace, dev_err)
+    if not (q.is_contiguous() and out.is_contiguous()):
+        raise ValueError("q and out must be contiguous")
+    if q.dtype != pool.dtype or out.dtype != pool.dtype:
+        raise ValueError("q/out dtype must match the pool")
+    T, Hq, D = q.shape
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    ws_ptr = _ptr(workspace)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    lib = _lib.load()
+    _lib.check(lib.pkv_extend_attn(ctypes.byref(pool.c), layer, q.data_ptr(), Hq,
+                                   ctypes.byref(table.c), table_idx.data_ptr(),
+                                   prefix_lens.data_ptr(), extend_lens.data_ptr(),
+                                   q_offsets.data_ptr(), extend_lens.shape[0], T,
+                                   int(max_extend_len), scale, out.data_ptr(), ws_ptr, ws_bytes,
+                                   _ptr(dev_err), _stream_ptr(stream)), "extend_attn")

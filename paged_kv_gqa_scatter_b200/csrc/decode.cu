@@ -1,0 +1,604 @@
+// Split-KV GQA decode attention over the paged pool.
+//
+// What it computes: "Mini-SGLang 完整剖析" (blog.rzhang-lab.cn/post/3) §1.2 --
+// decode runs one query token per request over that request's whole KV
+// history and is bound by memory bandwidth; §4.6.4 -- the history is found
+// through the token-granular page table, cache_seqlens being the total KV
+// length; §4.5.3 -- Hq/Hkv query heads share one KV head.
+//
+// Design (B200):
+//  * The concatenation of all requests' contexts is cut into gridDim.x equal
+//    token ranges, one per CTA of a persistent grid (one CTA per SM).  A range
+//    may hold the tail of one request, whole requests and the head of another;
+//    each (request, CTA) intersection is a "piece".  Equal ranges balance the
+//    HBM traffic across SMs exactly, whatever the length mix.
+//  * Warp 0 is the producer: for each stage of 16 tokens it translates the
+//    tokens' slots through the page table and issues one 1-D bulk copy
+//    (cp.async.bulk, the TMA's non-tensor form) per token and plane.  A token
+//    row holds all KV heads of the slot (2 KB for 8 heads x 128 x bf16), so
+//    every copy is a long contiguous read.  Stages live in a 3-deep ring of
+//    shared memory guarded by full/empty mbarriers.
+//  * Warps 1..Hkv are consumers, one per KV head.  Lane = (half, c): c picks
+//    8 consecutive dims, half picks even/odd tokens.  Scores for 8 tokens x G
+//    heads are reduced across the 16 lanes of a half with a transposing
+//    butterfly (each step halves the values a lane keeps), so the reduction
+//    costs about one shuffle per (token, head) instead of four.  Softmax runs
+//    in the log2 domain with exp2 and a lazily moved running max (the
+//    accumulators are rescaled only when the max grows by more than 2^8).
+//    PV accumulates with packed f32x2 FMAs.
+//  * A piece that covers a whole request writes the final output; other
+//    pieces write an un-normalised fp32 partial plus (max, sum) to the
+//    workspace and decode_combine_kernel merges them.
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "launch.h"
+
+namespace pkv {
+
+namespace {
+
+constexpr int kMaxBatch = 4096;
+constexpr int kStages = 3;
+constexpr int kMinTokensPerCta = 32;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+
+template <typename E>
+struct DecodeTraits;
+template <>
+struct DecodeTraits<__nv_bfloat16> {
+  static constexpr int kTokensPerStage = 16;
+};
+template <>
+struct DecodeTraits<float> {
+  static constexpr int kTokensPerStage = 8;
+};
+
+struct DecodeArgs {
+  const uint8_t* kbase;
+  const uint8_t* vbase;
+  int64_t slot_stride_bytes;
+  int64_t num_slots;
+  const int32_t* table;
+  int64_t table_rows, table_cols, table_stride;
+  int32_t page_size;
+  const int32_t* table_idx;
+  const int32_t* seq_lens;
+  int32_t batch;
+  const void* q;
+  void* out;
+  int32_t hq, hkv;
+  float scale_log2;
+  int32_t row_bytes;  // Hkv * 128 * esize
+  int32_t* ws_cum;    // [batch + 1]
+  int64_t* ws_per;    // [1]
+  float2* ws_ml;      // [(grid + batch) * hq]
+  float* ws_o;        // [(grid + batch) * hq * 128]
+  int32_t* err;
+};
+
+// Shared memory layout (bytes), identical on host and device.
+struct DecodeSmem {
+  int32_t scan_off, cum_off, psm_off, ring_off, stage_bytes, total;
+};
+
+constexpr int kMaxThreads = 32 * 9;
+
+__host__ __device__ inline DecodeSmem decode_smem_layout(int batch, int hkv, int row_bytes, int T,
+                                                         int G) {
+  DecodeSmem L;
+  int off = 2 * kStages * 8 + 16;  // full/empty barriers + abort flag
+  L.scan_off = off;
+  off += 4 * kMaxThreads;
+  L.cum_off = off;
+  off += 4 * (batch + 1);
+  off = (off + 15) & ~15;
+  L.psm_off = off;
+  off += 4 * hkv * T * G;
+  off = (off + 127) & ~127;
+  L.ring_off = off;
+  L.stage_bytes = 2 * T * row_bytes;
+  L.total = off + kStages * L.stage_bytes;
+  return L;
+}
+
+// Transposing butterfly over the 16 lanes of a half-warp.  On entry every lane
+// holds V partial sums v[0..V); on exit lane c holds the complete sums of
+// values (V/16)*c .. (V/16)*c + V/16 - 1 (V >= 16), or of value c >> (4 - log2 V)
+// (V < 16, lanes sharing a value hold the same sum).
+template <int V>
+__device__ __forceinline__ void transpose_reduce16(float (&v)[V], int c) {
+  int n = V;
+#pragma unroll
+  for (int off = 8; off >= 1; off >>= 1) {
+    if (n >= 2) {
+      const bool upper = (c & off) != 0;
+#pragma unroll
+      for (int k = 0; k < V / 2; ++k) {
+        if (k < n / 2) {
+          const float send = upper ? v[k] : v[k + n / 2];
+          const float keep = upper ? v[k + n / 2] : v[k];
+          v[k] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+        }
+      }
+      n >>= 1;
+    } else {
+      v[0] += __shfl_xor_sync(0xffffffffu, v[0], off);
+    }
+  }
+}
+
+template <typename E, int G>
+__global__ void __launch_bounds__(32 * 9, 1) decode_split_kernel(const DecodeArgs a) {
+  constexpr int T = DecodeTraits<E>::kTokensPerStage;
+  constexpr int SUB = (64 / G < T) ? 64 / G : T;  // tokens per softmax sub-step
+  constexpr int HALF = SUB / 2;                    // tokens per lane per sub-step
+  constexpr int V = HALF * G;                      // partial sums per lane
+  constexpr int NV = V >= 16 ? V / 16 : 1;         // complete sums per lane after reduce
+  constexpr int LPH = 16 / G;                      // lanes per head within a half
+  constexpr int ESZ = sizeof(E);
+  constexpr int kLog2V = V >= 16 ? 4 : (V == 8 ? 3 : (V == 4 ? 2 : (V == 2 ? 1 : 0)));
+
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int ncons = a.hkv;
+  const DecodeSmem L = decode_smem_layout(a.batch, a.hkv, a.row_bytes, T, G);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem);
+  uint64_t* empty = full + kStages;
+  volatile int32_t* abort_flag = reinterpret_cast<volatile int32_t*>(empty + kStages);
+  int32_t* cum = reinterpret_cast<int32_t*>(smem + L.cum_off);
+  float* psm = reinterpret_cast<float*>(smem + L.psm_off);
+  uint8_t* ring = smem + L.ring_off;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], ncons);
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+
+  // ---- plan: prefix sums of clamped context lengths -------------------------
+  const int B = a.batch;
+  const int nthr = blockDim.x;
+  {
+    int32_t* scan = reinterpret_cast<int32_t*>(smem + L.scan_off);
+    const int seg = (B + nthr - 1) / nthr;
+    const int r0 = min(B, static_cast<int>(threadIdx.x) * seg);
+    const int r1 = min(B, r0 + seg);
+    int32_t ssum = 0;
+    for (int r = r0; r < r1; ++r) {
+      int32_t n = a.seq_lens[r];
+      if (blockIdx.x == 0) {
+        if (n < 1) set_err(a.err, PKV_DEV_ERR_EMPTY_CONTEXT);
+        if (n > a.table_cols) set_err(a.err, PKV_DEV_ERR_TABLE_RANGE);
+      }
+      n = n < 0 ? 0 : (n > a.table_cols ? static_cast<int32_t>(a.table_cols) : n);
+      cum[r + 1] = n;
+      ssum += n;
+    }
+    scan[threadIdx.x] = ssum;
+    __syncthreads();
+    if (warp == 0) {
+      int32_t carry = 0;
+      for (int base = 0; base < nthr; base += 32) {
+        const int32_t x0 = (base + lane < nthr) ? scan[base + lane] : 0;
+        int32_t x = x0;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+          const int32_t y = __shfl_up_sync(0xffffffffu, x, off);
+          if (lane >= off) x += y;
+        }
+        if (base + lane < nthr) scan[base + lane] = carry + x - x0;
+        carry += __shfl_sync(0xffffffffu, x, 31);
+      }
+    }
+    __syncthreads();
+    int32_t run = scan[threadIdx.x];
+    for (int r = r0; r < r1; ++r) {
+      run += cum[r + 1];
+      cum[r + 1] = run;
+    }
+    if (threadIdx.x == 0) cum[0] = 0;
+    __syncthreads();
+  }
+  const int64_t total = cum[B];
+  int64_t per = (total + gridDim.x - 1) / gridDim.x;
+  if (per < kMinTokensPerCta) per = kMinTokensPerCta;
+  if (blockIdx.x == 0) {
+    for (int r = threadIdx.x; r <= B; r += nthr) a.ws_cum[r] = cum[r];
+    if (threadIdx.x == 0) a.ws_per[0] = per;
+  }
+  const int64_t lo = static_cast<int64_t>(blockIdx.x) * per;
+  const int64_t hi = min(total, lo + per);
+  if (lo >= hi) return;  // idle CTA (no barrier traffic started)
+  // First request whose range contains token lo: largest r with cum[r] <= lo.
+  int rfirst = 0;
+  {
+    int l = 0, h = B;  // invariant cum[l] <= lo
+    while (h - l > 1) {
+      const int m = (l + h) >> 1;
+      if (cum[m] <= lo) l = m; else h = m;
+    }
+    rfirst = l;
+  }
+
+  if (warp == 0) {
+    // =========================== producer ===================================
+    const uint64_t policy = policy_evict_first();
+    int64_t s = 0;  // stage counter
+    int last_use[kStages];
+#pragma unroll
+    for (int i = 0; i < kStages; ++i) last_use[i] = -1;
+    bool aborted = false;
+    for (int r = rfirst; r < B && cum[r] < hi && !aborted; ++r) {
+      const int64_t ja = max(lo, (int64_t)cum[r]) - cum[r];
+      const int64_t jb = min(hi, (int64_t)cum[r + 1]) - cum[r];
+      if (jb <= ja) continue;
+      const int32_t trow = a.table_idx[r];
+      const bool row_ok = trow >= 0 && trow < a.table_rows;
+      if (!row_ok && lane == 0) set_err(a.err, PKV_DEV_ERR_TABLE_RANGE);
+      const int32_t* rowp = a.table + (row_ok ? trow : 0) * a.table_stride;
+      for (int64_t j0 = ja; j0 < jb; j0 += T, ++s) {
+        const int slot_i = static_cast<int>(s % kStages);
+        const int use = static_cast<int>(s / kStages);
+        if (use >= 1) {
+          bool ok = true;
+          if (lane == 0) ok = mbar_wait(&empty[slot_i], (use - 1) & 1);
+          ok = __shfl_sync(0xffffffffu, ok, 0);
+          if (!ok || *abort_flag) {
+            if (!ok && lane == 0) set_err(a.err, PKV_DEV_ERR_TIMEOUT);
+            *abort_flag = 1;
+            aborted = true;
+            break;
+          }
+        }
+        uint8_t* kst = ring + slot_i * L.stage_bytes;
+        uint8_t* vst = kst + T * a.row_bytes;
+        const int64_t j = j0 + lane;
+        const bool in_piece = lane < T && j < jb;
+        int64_t slot = -1;
+        if (in_piece && row_ok) slot = token_slot(rowp, j, a.page_size, a.num_slots, a.err);
+        const bool load = in_piece && slot >= 0;
+        if (in_piece && !load) {
+          // Out-of-range entry: the row reads as zeros (error already flagged).
+          for (int b = 0; b < a.row_bytes; b += 16) {
+            *reinterpret_cast<uint4*>(kst + lane * a.row_bytes + b) = make_uint4(0, 0, 0, 0);
+            *reinterpret_cast<uint4*>(vst + lane * a.row_bytes + b) = make_uint4(0, 0, 0, 0);
+          }
+          // Later bulk copies (async proxy) may write these bytes again.
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        }
+        const unsigned nload = __popc(__ballot_sync(0xffffffffu, load));
+        __syncwarp();
+        if (lane == 0) mbar_arrive_expect_tx(&full[slot_i], nload * 2u * a.row_bytes);
+        __syncwarp();
+        if (load) {
+          bulk_g2s(kst + lane * a.row_bytes, a.kbase + slot * a.slot_stride_bytes, a.row_bytes,
+                   &full[slot_i], policy);
+          bulk_g2s(vst + lane * a.row_bytes, a.vbase + slot * a.slot_stride_bytes, a.row_bytes,
+                   &full[slot_i], policy);
+        }
+        last_use[slot_i] = use;
+      }
+    }
+    // Make sure no copy into this CTA's shared memory is still in flight.
+    if (lane == 0) {
+      for (int i = 0; i < kStages; ++i)
+        if (last_use[i] >= 0 && !mbar_wait(&full[i], last_use[i] & 1))
+          set_err(a.err, PKV_DEV_ERR_TIMEOUT);
+    }
+    return;
+  }
+
+  // ============================= consumers ==================================
+  const int g = warp - 1;  // KV head
+  if (g >= ncons) return;
+  const int c = lane & 15, half = lane >> 4;
+  float* pw = psm + g * SUB * G;  // this warp's p buffer [SUB][G]
+  const E* qbase = static_cast<const E*>(a.q);
+  E* obase = static_cast<E*>(a.out);
+  int64_t s = 0;
+  for (int r = rfirst; r < B && cum[r] < hi; ++r) {
+    const int64_t ja = max(lo, (int64_t)cum[r]) - cum[r];
+    const int64_t jb = min(hi, (int64_t)cum[r + 1]) - cum[r];
+    if (jb <= ja) continue;
+    const bool whole = cum[r] >= lo && cum[r + 1] <= hi;
+
+    float2 q2[G][4];
+#pragma unroll
+    for (int hh = 0; hh < G; ++hh) {
+      load8<E>(qbase + ((int64_t)r * a.hq + g * G + hh) * kHeadDim + 8 * c, q2[hh]);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        q2[hh][e].x *= a.scale_log2;
+        q2[hh][e].y *= a.scale_log2;
+      }
+    }
+    float2 o2[G][4];
+    float lsum[G];
+#pragma unroll
+    for (int hh = 0; hh < G; ++hh) {
+      lsum[hh] = 0.f;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) o2[hh][e] = make_float2(0.f, 0.f);
+    }
+    float m_run = -INFINITY;  // running max of this lane's head (log2 domain)
+
+    for (int64_t j0 = ja; j0 < jb; j0 += T, ++s) {
+      const int slot_i = static_cast<int>(s % kStages);
+      const int use = static_cast<int>(s / kStages);
+      bool ok = mbar_wait(&full[slot_i], use & 1);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok || *abort_flag) {
+        if (!ok && lane == 0) set_err(a.err, PKV_DEV_ERR_TIMEOUT);
+        *abort_flag = 1;
+        return;
+      }
+      const int ntok = static_cast<int>(min((int64_t)T, jb - j0));
+      const uint8_t* kst = ring + slot_i * L.stage_bytes;
+      const uint8_t* vst = kst + T * a.row_bytes;
+      const int head_off = (g * kHeadDim + 8 * c) * ESZ;
+
+#pragma unroll
+      for (int sub = 0; sub < T; sub += SUB) {
+        if (sub >= ntok) break;
+        // ---- scores: partial dot products over this lane's 8 dims ----------
+        float v[V];
+#pragma unroll
+        for (int i = 0; i < HALF; ++i) {
+          const int t = sub + 2 * i + half;
+          float2 k2[4];
+          load8<E>(reinterpret_cast<const E*>(kst + t * a.row_bytes + head_off), k2);
+#pragma unroll
+          for (int hh = 0; hh < G; ++hh) {
+            float2 acc = __fmul2_rn(k2[0], q2[hh][0]);
+            acc = __ffma2_rn(k2[1], q2[hh][1], acc);
+            acc = __ffma2_rn(k2[2], q2[hh][2], acc);
+            acc = __ffma2_rn(k2[3], q2[hh][3], acc);
+            v[hh * HALF + i] = acc.x + acc.y;
+          }
+        }
+        transpose_reduce16<V>(v, c);
+        // This lane now holds NV complete scores of head hl.
+        const int idx0 = V >= 16 ? NV * c : (c >> (4 - kLog2V));
+        const int hl = c / LPH;
+        float sc[NV];
+        float mx = -INFINITY;
+#pragma unroll
+        for (int k = 0; k < NV; ++k) {
+          const int idx = idx0 + k;
+          const int tt = 2 * (idx % HALF) + half;
+          sc[k] = (sub + tt < ntok) ? v[k] : -INFINITY;
+          mx = fmaxf(mx, sc[k]);
+        }
+#pragma unroll
+        for (int off = 1; off < LPH; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+        const bool need = mx > m_run + kRescaleThreshold;
+        float alpha = 1.f;
+        if (need) {
+          alpha = exp2f(m_run - mx);
+          m_run = mx;
+        }
+#pragma unroll
+        for (int k = 0; k < NV; ++k) {
+          const int idx = idx0 + k;
+          const int tt = 2 * (idx % HALF) + half;
+          pw[tt * G + hl] = exp2f(sc[k] - m_run);
+        }
+        if (__any_sync(0xffffffffu, need)) {
+#pragma unroll
+          for (int hh = 0; hh < G; ++hh) {
+            const float al = __shfl_sync(0xffffffffu, alpha, hh * LPH);
+            lsum[hh] *= al;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              o2[hh][e].x *= al;
+              o2[hh][e].y *= al;
+            }
+          }
+        }
+        __syncwarp();
+        // ---- PV ------------------------------------------------------------
+#pragma unroll
+        for (int i = 0; i < HALF; ++i) {
+          const int tt = 2 * i + half;
+          if (sub + tt < ntok) {
+            float2 v2[4];
+            load8<E>(reinterpret_cast<const E*>(vst + (sub + tt) * a.row_bytes + head_off), v2);
+#pragma unroll
+            for (int hh = 0; hh < G; ++hh) {
+              const float p = pw[tt * G + hh];
+              const float2 pp = make_float2(p, p);
+              lsum[hh] += p;
+#pragma unroll
+              for (int e = 0; e < 4; ++e) o2[hh][e] = __ffma2_rn(v2[e], pp, o2[hh][e]);
+            }
+          }
+        }
+        __syncwarp();
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[slot_i]);
+    }
+
+    // ---- finish the piece -----------------------------------------------------
+#pragma unroll
+    for (int hh = 0; hh < G; ++hh) {
+      lsum[hh] += __shfl_xor_sync(0xffffffffu, lsum[hh], 16);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        o2[hh][e].x += __shfl_xor_sync(0xffffffffu, o2[hh][e].x, 16);
+        o2[hh][e].y += __shfl_xor_sync(0xffffffffu, o2[hh][e].y, 16);
+      }
+    }
+    float mh[G];
+#pragma unroll
+    for (int hh = 0; hh < G; ++hh) mh[hh] = __shfl_sync(0xffffffffu, m_run, hh * LPH);
+#pragma unroll
+    for (int hh = 0; hh < G; ++hh) {
+      if ((G >= 2 ? (hh & 1) : 0) != half) continue;
+      const int h = g * G + hh;
+      if (whole) {
+        const float inv = lsum[hh] > 0.f ? 1.f / lsum[hh] : 0.f;
+        float f[8];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          f[2 * e] = o2[hh][e].x * inv;
+          f[2 * e + 1] = o2[hh][e].y * inv;
+        }
+        store8<E>(obase + ((int64_t)r * a.hq + h) * kHeadDim + 8 * c, f);
+      } else {
+        const int64_t id = static_cast<int64_t>(blockIdx.x) + r;
+        float* op = a.ws_o + (id * a.hq + h) * kHeadDim + 8 * c;
+        *reinterpret_cast<float4*>(op) = make_float4(o2[hh][0].x, o2[hh][0].y, o2[hh][1].x, o2[hh][1].y);
+        *reinterpret_cast<float4*>(op + 4) =
+            make_float4(o2[hh][2].x, o2[hh][2].y, o2[hh][3].x, o2[hh][3].y);
+        if (c == 0) a.ws_ml[id * a.hq + h] = make_float2(mh[hh], lsum[hh]);
+      }
+    }
+  }
+}
+
+// Merge the pieces of requests that spanned more than one CTA; zero the rows
+// of empty contexts.  One warp per (request, q head); lane owns 4 dims.
+template <typename E>
+__global__ void __launch_bounds__(128) decode_combine_kernel(
+    const int32_t* __restrict__ seq_lens, const int32_t* __restrict__ cum,
+    const int64_t* __restrict__ per_p, const float2* __restrict__ ml, const float* __restrict__ o,
+    int32_t hq, void* __restrict__ out) {
+  const int r = blockIdx.x;
+  const int h = blockIdx.y * 4 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (h >= hq) return;
+  E* dst = static_cast<E*>(out) + ((int64_t)r * hq + h) * kHeadDim + 4 * lane;
+  const int64_t c0 = cum[r], c1 = cum[r + 1];
+  if (seq_lens[r] < 1 || c1 <= c0) {
+    if constexpr (sizeof(E) == 2) {
+      *reinterpret_cast<uint2*>(dst) = make_uint2(0, 0);
+    } else {
+      *reinterpret_cast<float4*>(dst) = make_float4(0, 0, 0, 0);
+    }
+    return;
+  }
+  const int64_t per = *per_p;
+  const int64_t k_lo = c0 / per, k_hi = (c1 - 1) / per;
+  if (k_lo == k_hi) return;  // written by its only piece
+  float M = -INFINITY;
+  for (int64_t k = k_lo; k <= k_hi; ++k) M = fmaxf(M, ml[(k + r) * hq + h].x);
+  float4 acc = make_float4(0, 0, 0, 0);
+  float den = 0.f;
+  for (int64_t k = k_lo; k <= k_hi; ++k) {
+    const float2 st = ml[(k + r) * hq + h];
+    const float w = exp2f(st.x - M);
+    den += w * st.y;
+    const float4 x = *reinterpret_cast<const float4*>(o + ((k + r) * hq + h) * kHeadDim + 4 * lane);
+    acc.x += w * x.x;
+    acc.y += w * x.y;
+    acc.z += w * x.z;
+    acc.w += w * x.w;
+  }
+  const float inv = den > 0.f ? 1.f / den : 0.f;
+  if constexpr (sizeof(E) == 2) {
+    uint2 w;
+    w.x = pack_bf16x2(acc.x * inv, acc.y * inv);
+    w.y = pack_bf16x2(acc.z * inv, acc.w * inv);
+    *reinterpret_cast<uint2*>(dst) = w;
+  } else {
+    *reinterpret_cast<float4*>(dst) = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+  }
+}
+
+template <typename E, int G>
+cudaError_t launch_decode_t(const DecodeArgs& a, int grid, cudaStream_t s) {
+  constexpr int T = DecodeTraits<E>::kTokensPerStage;
+  const DecodeSmem L = decode_smem_layout(a.batch, a.hkv, a.row_bytes, T, G);
+  cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<E, G>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, L.total);
+  if (e != cudaSuccess) return e;
+  decode_split_kernel<E, G><<<grid, 32 * (1 + a.hkv), L.total, s>>>(a);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  dim3 cg(a.batch, (a.hq + 3) / 4);
+  decode_combine_kernel<E><<<cg, 128, 0, s>>>(a.seq_lens, a.ws_cum, a.ws_per, a.ws_ml, a.ws_o,
+                                              a.hq, a.out);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+int decode_grid_size() {
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  return sms;
+}
+
+size_t decode_workspace_bytes(int32_t batch, int32_t num_q_heads, int grid) {
+  const size_t pieces = static_cast<size_t>(grid) + static_cast<size_t>(batch);
+  size_t b = 0;
+  b += 16;                                               // per
+  b += ((static_cast<size_t>(batch) + 1) * 4 + 15) & ~size_t(15);  // cum
+  b += pieces * num_q_heads * sizeof(float2);            // (m, l)
+  b = (b + 15) & ~size_t(15);
+  b += pieces * num_q_heads * kHeadDim * sizeof(float);  // partial O
+  return b;
+}
+
+cudaError_t launch_decode(const PoolView& pool, const TableView& t, const void* q,
+                          int32_t num_q_heads, const int32_t* table_idx, const int32_t* seq_lens,
+                          int32_t batch, float scale, void* out, void* workspace, int grid,
+                          int32_t* err, cudaStream_t s) {
+  if (batch == 0) return cudaSuccess;
+  DecodeArgs a;
+  a.kbase = pool.k;
+  a.vbase = pool.v;
+  a.slot_stride_bytes = pool.slot_stride_bytes;
+  a.num_slots = pool.num_slots;
+  a.table = t.entries;
+  a.table_rows = t.rows;
+  a.table_cols = t.cols;
+  a.table_stride = t.row_stride;
+  a.page_size = pool.page_size;
+  a.table_idx = table_idx;
+  a.seq_lens = seq_lens;
+  a.batch = batch;
+  a.q = q;
+  a.out = out;
+  a.hq = num_q_heads;
+  a.hkv = pool.num_kv_heads;
+  a.scale_log2 = scale * kLog2e;
+  a.row_bytes = pool.num_kv_heads * kHeadDim * pool.esize;
+  uint8_t* w = static_cast<uint8_t*>(workspace);
+  a.ws_per = reinterpret_cast<int64_t*>(w);
+  w += 16;
+  a.ws_cum = reinterpret_cast<int32_t*>(w);
+  w += ((static_cast<size_t>(batch) + 1) * 4 + 15) & ~size_t(15);
+  const size_t pieces = static_cast<size_t>(grid) + static_cast<size_t>(batch);
+  a.ws_ml = reinterpret_cast<float2*>(w);
+  w += pieces * num_q_heads * sizeof(float2);
+  w = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(w) + 15) & ~uintptr_t(15));
+  a.ws_o = reinterpret_cast<float*>(w);
+  a.err = err;
+  const int G = num_q_heads / pool.num_kv_heads;
+  if (pool.dtype == PKV_DTYPE_BF16) {
+    switch (G) {
+      case 1: return launch_decode_t<__nv_bfloat16, 1>(a, grid, s);
+      case 2: return launch_decode_t<__nv_bfloat16, 2>(a, grid, s);
+      case 4: return launch_decode_t<__nv_bfloat16, 4>(a, grid, s);
+      case 8: return launch_decode_t<__nv_bfloat16, 8>(a, grid, s);
+    }
+  } else {
+    switch (G) {
+      case 1: return launch_decode_t<float, 1>(a, grid, s);
+      case 2: return launch_decode_t<float, 2>(a, grid, s);
+      case 4: return launch_decode_t<float, 4>(a, grid, s);
+      case 8: return launch_decode_t<float, 8>(a, grid, s);
+    }
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace pkv

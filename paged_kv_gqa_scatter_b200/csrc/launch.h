@@ -1,0 +1,62 @@
+// Host-side launchers of the pkv kernels (internal; the public ABI is include/pkv.h).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/pkv.h"
+
+namespace pkv {
+
+constexpr int kHeadDimHost = 128;
+
+struct PoolView {
+  const uint8_t* k;  // layer base (bytes)
+  const uint8_t* v;
+  uint8_t* k_mut;
+  uint8_t* v_mut;
+  int64_t slot_stride_bytes;
+  int64_t num_slots;
+  int32_t num_kv_heads;
+  int32_t page_size;
+  int32_t esize;  // element size in bytes
+  int32_t dtype;
+};
+
+struct TableView {
+  const int32_t* entries;
+  int64_t rows;
+  int64_t cols;
+  int64_t row_stride;
+};
+
+cudaError_t launch_store_kv(const PoolView& pool, const void* k, int64_t k_stride_bytes,
+                            const void* v, int64_t v_stride_bytes, const void* out_loc,
+                            bool loc_i64, int64_t n, int32_t* err, cudaStream_t s);
+
+cudaError_t launch_gather_kv(const PoolView& pool, const TableView& t, const int32_t* table_idx,
+                             const int32_t* seq_lens, const int64_t* row_offsets, int32_t batch,
+                             void* k_out, void* v_out, int32_t* err, cudaStream_t s);
+
+// Split-KV decode.
+size_t decode_workspace_bytes(int32_t batch, int32_t num_q_heads, int grid);
+int decode_grid_size();
+cudaError_t launch_decode(const PoolView& pool, const TableView& t, const void* q,
+                          int32_t num_q_heads, const int32_t* table_idx, const int32_t* seq_lens,
+                          int32_t batch, float scale, void* out, void* workspace, int grid,
+                          int32_t* err, cudaStream_t s);
+
+// Extend: tcgen05 path (bf16) and CUDA-core path (fp32 check build).
+cudaError_t launch_extend_tc(const PoolView& pool, const TableView& t, const void* q,
+                             int32_t num_q_heads, const int32_t* table_idx,
+                             const int32_t* prefix_lens, const int32_t* extend_lens,
+                             const int32_t* q_offsets, int32_t batch, int64_t total_q, int32_t max_extend,
+                             float scale, void* out, int32_t* err, cudaStream_t s);
+cudaError_t launch_extend_simt(const PoolView& pool, const TableView& t, const void* q,
+                               int32_t num_q_heads, const int32_t* table_idx,
+                               const int32_t* prefix_lens, const int32_t* extend_lens,
+                               const int32_t* q_offsets, int32_t batch, int64_t total_q, int32_t max_extend,
+                               float scale, void* out, int32_t* err, cudaStream_t s);
+
+}  // namespace pkv
