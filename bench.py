@@ -235,7 +235,7 @@ def run_decode(args, world, rank, local):
         wl = W.decode_qwen3_8b(num_pages=num_pages)
         layers = list(range(wl.pool.num_layers))
     else:
-        wl = W.decode_qwen3_06b()
+        wl = W.decode_qwen3_06b(num_layers=args.pool_layers, layer=min(13, args.pool_layers - 1))
         layers = [wl.layer]
     lib = _lib.load()
 
@@ -512,6 +512,8 @@ def main():
     ap.add_argument("--workload", default="decode-qwen3-0.6b",
                     choices=["decode-qwen3-0.6b", "decode-qwen3-8b"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--pool-layers", type=int, default=28,
+                    help="layers of the decode-qwen3-0.6b pool (28 as stated; fewer only for profiling)")
     ap.add_argument("--no-extend", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:

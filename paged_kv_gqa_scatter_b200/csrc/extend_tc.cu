@@ -1,15 +1,627 @@
-// Placeholder: routes bf16 extend to the CUDA-core kernel until the tensor-core kernel lands.
+// Causal extend attention on the tcgen05 tensor cores (bf16 in, fp32 accumulate).
+//
+// What it computes: "深入解析 mini-sglang" (yunpan.plus), chunked prefill -- a
+// chunk of a request attends to the KV its earlier chunks left in the pool,
+// reached through the request's page-table row, plus its own rows;
+// "Mini-SGLang 完整剖析" (blog.rzhang-lab.cn/post/3) §4.2.3 -- the chunk holds
+// extend_len = device_len - cached_len tokens after a cached prefix that may be
+// radix-shared (§1.4); §1.2 -- prefill is compute bound.  Query i of a chunk
+// sits at position prefix + i and sees keys 0 .. prefix + i; query head h
+// reads KV head h / (Hq/Hkv).
+//
+// Design (B200, one CTA per SM, 12 warps):
+//  * A CTA owns one (request, KV head, 2 x 128 query rows) block.  Rows are
+//    (token, query head of the group) pairs, token-major, so the G query heads
+//    sharing a KV head form the M dimension of one MMA and every K/V tile is
+//    used by 256 rows.
+//  * warp 0 -- loads: the two Q tiles once (3-D TMA boxes [tokens][G heads][64
+//    dims] with the 128-byte swizzle), then for each 128-key tile it
+//    translates the keys' slots through the page table and gathers the K and V
+//    rows with TMA tile::gather4 (4 pool rows per copy, 128-byte swizzle) into
+//    a 2-stage ring.  The gathered layout is directly the UMMA operand layout:
+//    K-major for K (B of Q K^T), MN-major for V (B of P V).
+//  * warp 1 -- MMA issue (one thread): S_i = Q_i K^T into TMEM (M=128, N=128,
+//    K=16 steps), then O_i += P_i V with P_i read from TMEM.  Issue order
+//    PV_0(j), QK_0(j+1), PV_1(j), QK_1(j+1) lets softmax of one Q tile run
+//    while the tensor core works on the other.  Completion is signalled with
+//    tcgen05.commit to mbarriers.  The warp also allocates / frees TMEM.
+//  * warps 4-7 and 8-11 -- softmax for Q tile 0 and 1: one thread per row,
+//    tcgen05.ld of its S row, log2-domain online softmax with a lazily moved
+//    max (O rescaled in TMEM only when the max grows by more than 2^8), P
+//    written back over S as packed bf16 with tcgen05.st; at the end O / l is
+//    read from TMEM and stored as bf16.
+//  * TMEM (512 columns): S_0, S_1, O_0, O_1, 128 fp32 columns each; P_i
+//    occupies the first 64 columns of S_i.
+//  * Every mbarrier wait is bounded (about one second); on a timeout the CTA
+//    records PKV_DEV_ERR_TIMEOUT, drains its copies and MMAs, frees TMEM and
+//    returns.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
 #include "launch.h"
 
 namespace pkv {
 
-cudaError_t launch_extend_tc(const PoolView& pool, const TableView& t, const void* q,
-                             int32_t num_q_heads, const int32_t* table_idx,
-                             const int32_t* prefix_lens, const int32_t* extend_lens,
+namespace {
+
+constexpr int kRowsPerTile = 128;
+constexpr int kKeysPerTile = 128;
+constexpr int kQTiles = 2;
+constexpr int kKvStages = 2;
+constexpr int kHalfBytes = 128 * 128;     // 128 rows x 64 bf16 (one swizzle column block)
+constexpr int kTileBytes = 2 * kHalfBytes;  // 128 rows x 128 bf16
+constexpr int kThreads = 384;
+
+// Shared memory map (offsets from a 1024-byte aligned base).
+constexpr int kOffQ = 0;
+constexpr int kOffK = kOffQ + kQTiles * kTileBytes;
+constexpr int kOffV = kOffK + kKvStages * kTileBytes;
+constexpr int kOffBar = kOffV + kKvStages * kTileBytes;
+constexpr int kNumBars = 16;
+constexpr int kOffMisc = kOffBar + kNumBars * 8;
+constexpr int kSmemBytes = kOffMisc + 64 + 1024;  // + slack for manual 1024-byte alignment
+
+// Barrier indices.
+constexpr int kBarQFull = 0;
+constexpr int kBarKFull = 1;    // +stage
+constexpr int kBarKEmpty = 3;   // +stage
+constexpr int kBarVFull = 5;    // +stage
+constexpr int kBarVEmpty = 7;   // +stage
+constexpr int kBarSFull = 9;    // +q tile
+constexpr int kBarPReady = 11;  // +q tile
+constexpr int kBarOFinal = 13;
+constexpr int kBarDrain = 14;
+
+// TMEM columns.
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColS = 0;    // + 128 * tile
+constexpr uint32_t kColO = 256;  // + 128 * tile
+
+constexpr float kRescaleThreshold = 8.0f;
+
+struct ExtendTcArgs {
+  const int32_t* table;
+  int64_t table_rows, table_cols, table_stride;
+  int32_t page_size;
+  int64_t num_slots;
+  const int32_t* table_idx;
+  const int32_t* prefix_lens;
+  const int32_t* extend_lens;
+  const int32_t* q_offsets;
+  int64_t total_q;
+  int32_t max_extend;
+  __nv_bfloat16* out;
+  int32_t hq, hkv;
+  float scale_log2;
+  int32_t* err;
+};
+
+// ---- PTX wrappers -----------------------------------------------------------
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, int c0, int c1, int c2,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* map, int col, int r0, int r1,
+                                            int r2, int r3, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(col), "r"(r0), "r"(r1), "r"(r2), "r"(r3),
+      "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// SMEM matrix descriptor: 128-byte swizzle, sm_100 version field.
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((addr >> 4) & 0x3FFF);
+  d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFF) << 16;
+  d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFF) << 32;
+  d |= static_cast<uint64_t>(1) << 46;   // version
+  d |= static_cast<uint64_t>(2) << 61;   // SWIZZLE_128B
+  return d;
+}
+
+// Instruction descriptor, kind::f16: bf16 A/B, fp32 D, M = 128, N = 128.
+constexpr uint32_t kIdescBase = (1u << 4) | (1u << 7) | (1u << 10) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
+constexpr uint32_t kIdescQK = kIdescBase;              // A K-major, B K-major
+constexpr uint32_t kIdescPV = kIdescBase | (1u << 16);  // B (V) MN-major
+
+__device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                       uint32_t accum) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accum)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                       uint32_t accum) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accum)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32"
+      " {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15,"
+      " %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]),
+        "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]),
+        "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0],"
+      " {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16,"
+      " %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+      "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+      "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+      "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
+      "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+      "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+      "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])), "r"(__float_as_uint(v[17])),
+      "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])), "r"(__float_as_uint(v[20])),
+      "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])), "r"(__float_as_uint(v[23])),
+      "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])),
+      "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])),
+      "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&w)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0],"
+      " {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+      "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7]),
+      "r"(w[8]), "r"(w[9]), "r"(w[10]), "r"(w[11]), "r"(w[12]), "r"(w[13]), "r"(w[14]), "r"(w[15])
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_st() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// ---- the kernel ---------------------------------------------------------------
+template <int G>
+__global__ void __launch_bounds__(kThreads, 1)
+    extend_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
+                     const __grid_constant__ CUtensorMap vmap, const ExtendTcArgs a) {
+  constexpr int TQ = kRowsPerTile / G;  // tokens per Q tile
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
+  volatile int32_t* abort_flag = reinterpret_cast<volatile int32_t*>(smem + kOffMisc + 16);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int r = blockIdx.z, g = blockIdx.y;
+  const int qb = static_cast<int>(gridDim.x) - 1 - static_cast<int>(blockIdx.x);  // heaviest first
+
+  // ---- block-uniform work description (identical in every thread) ---------
+  const int32_t p = a.prefix_lens[r], e = a.extend_lens[r];
+  const int64_t qbase = a.q_offsets[r];
+  if (p < 0 || e < 0 || qbase < 0 || qbase + e > a.total_q) {
+    if (threadIdx.x == 0 && blockIdx.x == 0 && g == 0) set_err(a.err, PKV_DEV_ERR_BAD_LENGTH);
+    return;
+  }
+  if (e > a.max_extend && threadIdx.x == 0 && blockIdx.x == 0 && g == 0)
+    set_err(a.err, PKV_DEV_ERR_BAD_LENGTH);
+  const int i0 = qb * (kQTiles * TQ);
+  if (i0 >= e) return;
+  const int32_t trow = a.table_idx[r];
+  const bool row_ok = trow >= 0 && trow < a.table_rows;
+  int64_t kv_end = static_cast<int64_t>(p) + min(e, i0 + kQTiles * TQ);
+  if (kv_end > a.table_cols) {
+    if (threadIdx.x == 0) set_err(a.err, PKV_DEV_ERR_TABLE_RANGE);
+    kv_end = a.table_cols;
+  }
+  if (!row_ok && threadIdx.x == 0) set_err(a.err, PKV_DEV_ERR_TABLE_RANGE);
+  const int ntiles = static_cast<int>((kv_end + kKeysPerTile - 1) / kKeysPerTile);
+
+  // ---- setup: barriers and TMEM ------------------------------------------------
+  if (threadIdx.x == 0) {
+    mbar_init(&bars[kBarQFull], 1);
+    for (int s = 0; s < kKvStages; ++s) {
+      mbar_init(&bars[kBarKFull + s], 1);
+      mbar_init(&bars[kBarKEmpty + s], 1);
+      mbar_init(&bars[kBarVFull + s], 1);
+      mbar_init(&bars[kBarVEmpty + s], 1);
+    }
+    for (int i = 0; i < kQTiles; ++i) {
+      mbar_init(&bars[kBarSFull + i], 1);
+      mbar_init(&bars[kBarPReady + i], 128);
+    }
+    mbar_init(&bars[kBarOFinal], 1);
+    mbar_init(&bars[kBarDrain], 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  uint8_t* sQ = smem + kOffQ;
+  uint8_t* sK = smem + kOffK;
+  uint8_t* sV = smem + kOffV;
+
+  if (warp == 0) {
+    // ============================ loads =======================================
+    const int32_t* rowp = a.table + (row_ok ? trow : 0) * a.table_stride;
+    if (lane == 0) {
+      mbar_arrive_expect_tx(&bars[kBarQFull], kQTiles * kTileBytes);
+      for (int i = 0; i < kQTiles; ++i)
+        for (int h = 0; h < 2; ++h)
+          tma_load_3d(sQ + i * kTileBytes + h * kHalfBytes, &qmap, h * 64, g * G,
+                      static_cast<int>(qbase + i0 + i * TQ), &bars[kBarQFull]);
+    }
+    // A masked key reads the request's first key row (finite, part of its context).
+    int32_t dummy = 0;
+    if (row_ok) {
+      const int64_t s0 = token_slot(rowp, 0, a.page_size, a.num_slots, nullptr);
+      dummy = s0 >= 0 ? static_cast<int32_t>(s0) : 0;
+    }
+    int k_last_use[kKvStages] = {-1, -1};
+    int v_last_use[kKvStages] = {-1, -1};
+    bool ok = true;
+    for (int j = 0; j < ntiles && ok; ++j) {
+      const int st = j & 1, use = j >> 1;
+      int rows[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int64_t key = static_cast<int64_t>(j) * kKeysPerTile + lane * 4 + u;
+        int64_t s = -1;
+        if (key < kv_end && row_ok) s = token_slot(rowp, key, a.page_size, a.num_slots, a.err);
+        rows[u] = s >= 0 ? static_cast<int32_t>(s) : dummy;
+      }
+      if (use >= 1) {
+        bool w = true;
+        if (lane == 0) w = mbar_wait(&bars[kBarKEmpty + st], (use - 1) & 1);
+        w = __shfl_sync(0xffffffffu, w, 0);
+        if (__any_sync(0xffffffffu, !w || *abort_flag != 0)) { ok = false; break; }
+      }
+      if (lane == 0) mbar_arrive_expect_tx(&bars[kBarKFull + st], kTileBytes);
+      __syncwarp();
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+        tma_gather4(sK + st * kTileBytes + h * kHalfBytes + lane * 4 * 128, &kmap, g * 128 + h * 64,
+                    rows[0], rows[1], rows[2], rows[3], &bars[kBarKFull + st]);
+      k_last_use[st] = use;
+      if (use >= 1) {
+        bool w = true;
+        if (lane == 0) w = mbar_wait(&bars[kBarVEmpty + st], (use - 1) & 1);
+        w = __shfl_sync(0xffffffffu, w, 0);
+        if (__any_sync(0xffffffffu, !w || *abort_flag != 0)) { ok = false; break; }
+      }
+      if (lane == 0) mbar_arrive_expect_tx(&bars[kBarVFull + st], kTileBytes);
+      __syncwarp();
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+        tma_gather4(sV + st * kTileBytes + h * kHalfBytes + lane * 4 * 128, &vmap, g * 128 + h * 64,
+                    rows[0], rows[1], rows[2], rows[3], &bars[kBarVFull + st]);
+      v_last_use[st] = use;
+    }
+    if (!ok && lane == 0) {
+      set_err(a.err, PKV_DEV_ERR_TIMEOUT);
+      *abort_flag = 1;
+    }
+    // Every copy issued into this CTA's shared memory must land before exit.
+    if (lane == 0) {
+      if (!mbar_wait(&bars[kBarQFull], 0)) set_err(a.err, PKV_DEV_ERR_TIMEOUT);
+      for (int s = 0; s < kKvStages; ++s) {
+        if (k_last_use[s] >= 0 && !mbar_wait(&bars[kBarKFull + s], k_last_use[s] & 1))
+          set_err(a.err, PKV_DEV_ERR_TIMEOUT);
+        if (v_last_use[s] >= 0 && !mbar_wait(&bars[kBarVFull + s], v_last_use[s] & 1))
+          set_err(a.err, PKV_DEV_ERR_TIMEOUT);
+      }
+    }
+  } else if (warp == 1) {
+    // ============================ MMA issue ===================================
+    if (lane == 0) {
+      const uint32_t q_addr = smem_u32(sQ);
+      const uint32_t k_addr = smem_u32(sK);
+      const uint32_t v_addr = smem_u32(sV);
+      bool ok = mbar_wait(&bars[kBarQFull], 0);
+      auto issue_qk = [&](int i, int st) {
+        const uint32_t d = tmem + kColS + 128 * i;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
+          const uint64_t ad = smem_desc(q_addr + i * kTileBytes + off, 16, 1024);
+          const uint64_t bd = smem_desc(k_addr + st * kTileBytes + off, 16, 1024);
+          mma_ss(d, ad, bd, kIdescQK, kk > 0 ? 1u : 0u);
+        }
+      };
+      auto issue_pv = [&](int i, int st, bool first) {
+        const uint32_t d = tmem + kColO + 128 * i;
+        const uint32_t pa = tmem + kColS + 128 * i;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint64_t bd = smem_desc(v_addr + st * kTileBytes + kk * 2048, kHalfBytes, 1024);
+          mma_ts(d, pa + kk * 8, bd, kIdescPV, (first && kk == 0) ? 0u : 1u);
+        }
+      };
+      if (ok) ok = mbar_wait(&bars[kBarKFull + 0], 0);
+      if (ok) {
+        tc_fence_after();
+        issue_qk(0, 0);
+        mma_commit(&bars[kBarSFull + 0]);
+        issue_qk(1, 0);
+        mma_commit(&bars[kBarSFull + 1]);
+        mma_commit(&bars[kBarKEmpty + 0]);
+      }
+      for (int j = 0; j < ntiles && ok; ++j) {
+        const int st = j & 1, use = j >> 1;
+        const int st1 = (j + 1) & 1, use1 = (j + 1) >> 1;
+        ok = mbar_wait(&bars[kBarVFull + st], use & 1) && mbar_wait(&bars[kBarPReady + 0], j & 1);
+        if (!ok || *abort_flag) break;
+        tc_fence_after();
+        issue_pv(0, st, j == 0);
+        if (j + 1 < ntiles) {
+          ok = mbar_wait(&bars[kBarKFull + st1], use1 & 1);
+          if (!ok) break;
+          tc_fence_after();
+          issue_qk(0, st1);
+          mma_commit(&bars[kBarSFull + 0]);
+        }
+        ok = mbar_wait(&bars[kBarPReady + 1], j & 1);
+        if (!ok || *abort_flag) break;
+        tc_fence_after();
+        issue_pv(1, st, j == 0);
+        mma_commit(&bars[kBarVEmpty + st]);
+        if (j + 1 < ntiles) {
+          issue_qk(1, st1);
+          mma_commit(&bars[kBarSFull + 1]);
+          mma_commit(&bars[kBarKEmpty + st1]);
+        }
+      }
+      if (!ok) {
+        set_err(a.err, PKV_DEV_ERR_TIMEOUT);
+        *abort_flag = 1;
+      }
+      // Final commit: O complete (or, after an abort, every issued MMA retired).
+      mma_commit(&bars[kBarOFinal]);
+      if (!mbar_wait(&bars[kBarOFinal], 0)) set_err(a.err, PKV_DEV_ERR_TIMEOUT);
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ============================ softmax + epilogue ==========================
+    const int i = (warp - 4) >> 2;   // Q tile
+    const int wq = warp & 3;         // TMEM lane quadrant
+    const int m = wq * 32 + lane;    // row within the tile
+    const int tq = m / G, hh = m % G;
+    const int tok = i0 + i * TQ + tq;
+    const bool valid = tok < e;
+    const int64_t lim = valid ? static_cast<int64_t>(p) + tok + 1 : 1;  // keys < lim visible
+    const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
+    const uint32_t s_addr = tmem + lane_base + kColS + 128 * i;
+    const uint32_t o_addr = tmem + lane_base + kColO + 128 * i;
+    float m_run = -INFINITY, l_run = 0.f;
+    bool ok = true;
+    for (int j = 0; j < ntiles; ++j) {
+      const bool w = mbar_wait(&bars[kBarSFull + i], j & 1);
+      if (__any_sync(0xffffffffu, !w || *abort_flag != 0)) { ok = false; break; }
+      tc_fence_after();
+      const int64_t kb = static_cast<int64_t>(j) * kKeysPerTile;
+      const bool full_tile = kb + kKeysPerTile <= lim;
+      float mx = -INFINITY;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        float v[32];
+        tmem_ld32(s_addr + c * 32, v);
+#pragma unroll
+        for (int u = 0; u < 32; ++u) {
+          const bool vis = full_tile || (kb + c * 32 + u < lim);
+          mx = vis ? fmaxf(mx, v[u]) : mx;
+        }
+      }
+      mx *= a.scale_log2;
+      const bool need = mx > m_run + kRescaleThreshold;
+      if (j > 0 && __any_sync(0xffffffffu, need)) {
+        const float alpha = need ? exp2f(m_run - mx) : 1.f;
+        l_run *= alpha;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          float o[32];
+          tmem_ld32(o_addr + c * 32, o);
+#pragma unroll
+          for (int u = 0; u < 32; ++u) o[u] *= alpha;
+          tmem_st32(o_addr + c * 32, o);
+        }
+        tmem_wait_st();
+      }
+      if (need) m_run = mx;
+      const float neg_m = -m_run;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        float v[32];
+        tmem_ld32(s_addr + c * 32, v);
+        uint32_t w16[16];
+#pragma unroll
+        for (int u = 0; u < 32; u += 2) {
+          const bool vis0 = full_tile || (kb + c * 32 + u < lim);
+          const bool vis1 = full_tile || (kb + c * 32 + u + 1 < lim);
+          const float p0 = vis0 ? exp2f(fmaf(v[u], a.scale_log2, neg_m)) : 0.f;
+          const float p1 = vis1 ? exp2f(fmaf(v[u + 1], a.scale_log2, neg_m)) : 0.f;
+          l_run += p0 + p1;
+          w16[u >> 1] = pack_bf16x2(p0, p1);
+        }
+        tmem_st16(s_addr + c * 16, w16);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&bars[kBarPReady + i]);
+    }
+    if (!ok && lane == 0) {
+      set_err(a.err, PKV_DEV_ERR_TIMEOUT);
+      *abort_flag = 1;
+    }
+    bool w = mbar_wait(&bars[kBarOFinal], 0);
+    w = __all_sync(0xffffffffu, w);
+    tc_fence_after();
+    if (w && ok) {
+      const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+      __nv_bfloat16* dst = a.out + ((qbase + tok) * a.hq + g * G + hh) * kHeadDim;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        float o[32];
+        tmem_ld32(o_addr + c * 32, o);
+        if (valid) {
+#pragma unroll
+          for (int u = 0; u < 32; u += 8) {
+            uint4 pk;
+            pk.x = pack_bf16x2(o[u] * inv, o[u + 1] * inv);
+            pk.y = pack_bf16x2(o[u + 2] * inv, o[u + 3] * inv);
+            pk.z = pack_bf16x2(o[u + 4] * inv, o[u + 5] * inv);
+            pk.w = pack_bf16x2(o[u + 6] * inv, o[u + 7] * inv);
+            *reinterpret_cast<uint4*>(dst + c * 32 + u) = pk;
+          }
+        }
+      }
+    } else if (lane == 0) {
+      set_err(a.err, PKV_DEV_ERR_TIMEOUT);
+    }
+  }
+
+  // ---- teardown: every role is done with TMEM --------------------------------
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols)
+                 : "memory");
+  }
+}
+
+// ---- host side ----------------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (fn == nullptr) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+bool make_row_map(CUtensorMap* map, const void* base, int64_t row_elems, int64_t rows, int64_t row_stride_bytes) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(row_elems), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(row_stride_bytes)};
+  cuuint32_t box[2] = {64, 1};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool make_q_map(CUtensorMap* map, const void* q, int32_t hq, int64_t total_q, int G) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(hq), static_cast<cuuint64_t>(total_q)};
+  cuuint64_t strides[2] = {128 * 2, static_cast<cuuint64_t>(hq) * 128 * 2};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(G), static_cast<cuuint32_t>(128 / G)};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(q), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int G>
+cudaError_t launch_g(const CUtensorMap& qm, const CUtensorMap& km, const CUtensorMap& vm, const ExtendTcArgs& a,
+                     int32_t batch, int32_t max_extend, cudaStream_t s) {
+  constexpr int TQ = kRowsPerTile / G;
+  const int nqb = (max_extend + kQTiles * TQ - 1) / (kQTiles * TQ);
+  cudaError_t e = cudaFuncSetAttribute(extend_tc_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  if (e != cudaSuccess) return e;
+  dim3 grid(nqb, a.hkv, batch);
+  extend_tc_kernel<G><<<grid, kThreads, kSmemBytes, s>>>(qm, km, vm, a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_extend_tc(const PoolView& pool, const TableView& t, const void* q, int32_t num_q_heads,
+                             const int32_t* table_idx, const int32_t* prefix_lens, const int32_t* extend_lens,
                              const int32_t* q_offsets, int32_t batch, int64_t total_q, int32_t max_extend,
                              float scale, void* out, int32_t* err, cudaStream_t s) {
-  return launch_extend_simt(pool, t, q, num_q_heads, table_idx, prefix_lens, extend_lens,
-                            q_offsets, batch, total_q, max_extend, scale, out, err, s);
+  if (batch == 0 || max_extend == 0 || total_q == 0) return cudaSuccess;
+  const int G = num_q_heads / pool.num_kv_heads;
+  CUtensorMap qm, km, vm;
+  const int64_t row_elems = static_cast<int64_t>(pool.num_kv_heads) * kHeadDimHost;
+  if (!make_q_map(&qm, q, num_q_heads, total_q, G) ||
+      !make_row_map(&km, pool.k, row_elems, pool.num_slots, pool.slot_stride_bytes) ||
+      !make_row_map(&vm, pool.v, row_elems, pool.num_slots, pool.slot_stride_bytes))
+    return cudaErrorInvalidValue;
+  ExtendTcArgs a;
+  a.table = t.entries;
+  a.table_rows = t.rows;
+  a.table_cols = t.cols;
+  a.table_stride = t.row_stride;
+  a.page_size = pool.page_size;
+  a.num_slots = pool.num_slots;
+  a.table_idx = table_idx;
+  a.prefix_lens = prefix_lens;
+  a.extend_lens = extend_lens;
+  a.q_offsets = q_offsets;
+  a.total_q = total_q;
+  a.max_extend = max_extend;
+  a.out = static_cast<__nv_bfloat16*>(out);
+  a.hq = num_q_heads;
+  a.hkv = pool.num_kv_heads;
+  a.scale_log2 = scale * kLog2e;
+  a.err = err;
+  switch (G) {
+    case 1: return launch_g<1>(qm, km, vm, a, batch, max_extend, s);
+    case 2: return launch_g<2>(qm, km, vm, a, batch, max_extend, s);
+    case 4: return launch_g<4>(qm, km, vm, a, batch, max_extend, s);
+    case 8: return launch_g<8>(qm, km, vm, a, batch, max_extend, s);
+  }
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace pkv
