@@ -198,6 +198,35 @@ int pkv_decode_attn(const pkv_pool* pool, int32_t layer, const void* q, int32_t 
                     pkv_stream_t stream);
 
 /*
+ * decode_attn_noalloc -- the same decode as pkv_decode_attn for callers that
+ * cannot allocate device memory.  The pages have no counterpart to this call.
+ *
+ * Who needs it: an engine that gives almost all free device memory to its KV
+ * pool when it starts has no room left to allocate a workspace, and code
+ * hosted by a framework that owns every device allocation may have no way to
+ * allocate at all.  This call takes the same arguments as pkv_decode_attn
+ * minus the workspace; its scratch is a fixed 16 MiB array inside the library
+ * (pkv_decode_noalloc_max_scratch_bytes()), present on every device that
+ * loads the library until the process exits.
+ *
+ * Limits and behaviour:
+ *  - Returns PKV_ERR_TOO_LARGE, launching nothing, when
+ *    pkv_decode_workspace_bytes(batch, num_q_heads) exceeds that size.
+ *  - The first call on each device (with it current) looks up the array's
+ *    device address and caches it; make that first call outside any stream
+ *    capture.
+ *  - All calls on a device share the array: calls that can overlap on the GPU
+ *    (unordered streams) race; calls ordered on one stream are safe.  Nothing
+ *    in the array needs to start at zero.
+ *  - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ */
+size_t pkv_decode_noalloc_max_scratch_bytes(void);
+int pkv_decode_attn_noalloc(const pkv_pool* pool, int32_t layer, const void* q,
+                            int32_t num_q_heads, const pkv_page_table* table,
+                            const int32_t* table_idx, const int32_t* seq_lens, int32_t batch,
+                            float scale, void* out, int32_t* dev_err, pkv_stream_t stream);
+
+/*
  * extend_attn [P4 chunked prefill: every chunk of a request uses the same
  * table row and reuses the KV of the chunks before it; P5 §4.2.3: a request
  * has cached_len (its prefix, possibly radix-shared) and extend_len =

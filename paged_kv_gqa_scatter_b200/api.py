@@ -145,6 +145,29 @@ def decode_attn(pool: KVPool, layer: int, q: torch.Tensor, table: PageTable,
                                    _stream_ptr(stream)), "decode_attn")
 
 
+def decode_attn_noalloc(pool: KVPool, layer: int, q: torch.Tensor, table: PageTable,
+                        table_idx: torch.Tensor, seq_lens: torch.Tensor, out: torch.Tensor,
+                        scale: Optional[float] = None, dev_err: Optional[torch.Tensor] = None,
+                        stream=None) -> None:
+    """pkv_decode_attn_noalloc: decode_attn without a workspace, for callers that
+    cannot allocate device memory.  Its scratch is a fixed array inside the
+    library shared by every call on the device, so calls that may overlap on
+    the GPU must not be issued; the first call on a device should happen
+    outside stream capture."""
+    _require_cuda(q, table_idx, seq_lens, out, dev_err)
+    if not (q.is_contiguous() and out.is_contiguous()):
+        raise ValueError("q and out must be contiguous")
+    if q.dtype != pool.dtype or out.dtype != pool.dtype:
+        raise ValueError("q/out dtype must match the pool")
+    B, Hq, D = q.shape
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    lib = _lib.load()
+    _lib.check(lib.pkv_decode_attn_noalloc(ctypes.byref(pool.c), layer, q.data_ptr(), Hq,
+                                           ctypes.byref(table.c), table_idx.data_ptr(),
+                                           seq_lens.data_ptr(), B, scale, out.data_ptr(),
+                                           _ptr(dev_err), _stream_ptr(stream)), "decode_attn_noalloc")
+
+
 def extend_workspace_bytes(batch: int, num_q_heads: int, total_q: int) -> int:
     return int(_lib.load().pkv_extend_workspace_bytes(batch, num_q_heads, total_q))
 
