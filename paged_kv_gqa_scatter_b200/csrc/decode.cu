@@ -140,6 +140,8 @@ __global__ void __launch_bounds__(32 * 9, 1) decode_split_kernel(const DecodeArg
   constexpr int kLog2V = V >= 16 ? 4 : (V == 8 ? 3 : (V == 4 ? 2 : (V == 2 ? 1 : 0)));
 
   extern __shared__ __align__(128) uint8_t smem[];
+  // Let the combine kernel be scheduled early; it waits for this grid anyway.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int ncons = a.hkv;
   const DecodeSmem L = decode_smem_layout(a.batch, a.hkv, a.row_bytes, T, G);
@@ -226,62 +228,122 @@ __global__ void __launch_bounds__(32 * 9, 1) decode_split_kernel(const DecodeArg
 
   if (warp == 0) {
     // =========================== producer ===================================
+    // Page-table entries are loaded two stages ahead of the copies that use
+    // them, so the dependent table read overlaps the wait for a free stage.
     const uint64_t policy = policy_evict_first();
-    int64_t s = 0;  // stage counter
+    struct Cursor {
+      int r;
+      int64_t j0, jb;
+      const int32_t* rowp;
+      bool row_ok;
+    };
+    // First non-empty piece at or after request rr.
+    auto piece_start = [&](int rr, Cursor& c) -> bool {
+      for (; rr < B && cum[rr] < hi; ++rr) {
+        const int64_t ja = max(lo, (int64_t)cum[rr]) - cum[rr];
+        const int64_t jb = min(hi, (int64_t)cum[rr + 1]) - cum[rr];
+        if (jb > ja) {
+          const int32_t trow = a.table_idx[rr];
+          c.row_ok = trow >= 0 && trow < a.table_rows;
+          if (!c.row_ok && lane == 0) set_err(a.err, PKV_DEV_ERR_TABLE_RANGE);
+          c.rowp = a.table + (c.row_ok ? trow : 0) * a.table_stride;
+          c.r = rr;
+          c.j0 = ja;
+          c.jb = jb;
+          return true;
+        }
+      }
+      return false;
+    };
+    auto advance = [&](Cursor& c) -> bool {
+      if (c.j0 + T < c.jb) {
+        c.j0 += T;
+        return true;
+      }
+      return piece_start(c.r + 1, c);
+    };
+    // This lane's raw table entry for a stage (the slot is derived at use).
+    auto lookup = [&](const Cursor& c, bool have) -> int32_t {
+      const int64_t j = c.j0 + lane;
+      if (!have || lane >= T || j >= c.jb || !c.row_ok) return 0;
+      return a.page_size == 1 ? c.rowp[j] : c.rowp[(j / a.page_size) * a.page_size];
+    };
+    Cursor c0{}, c1{}, c2{};
+    bool h0 = piece_start(rfirst, c0);
+    int32_t e0 = lookup(c0, h0);
+    c1 = c0;
+    bool h1 = h0 && advance(c1);
+    int32_t e1 = lookup(c1, h1);
+    c2 = c1;
+    bool h2 = h1 && advance(c2);
+    // Rows written by the preceding store_kv must be visible before any copy.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     int last_use[kStages];
 #pragma unroll
     for (int i = 0; i < kStages; ++i) last_use[i] = -1;
-    bool aborted = false;
-    for (int r = rfirst; r < B && cum[r] < hi && !aborted; ++r) {
-      const int64_t ja = max(lo, (int64_t)cum[r]) - cum[r];
-      const int64_t jb = min(hi, (int64_t)cum[r + 1]) - cum[r];
-      if (jb <= ja) continue;
-      const int32_t trow = a.table_idx[r];
-      const bool row_ok = trow >= 0 && trow < a.table_rows;
-      if (!row_ok && lane == 0) set_err(a.err, PKV_DEV_ERR_TABLE_RANGE);
-      const int32_t* rowp = a.table + (row_ok ? trow : 0) * a.table_stride;
-      for (int64_t j0 = ja; j0 < jb; j0 += T, ++s) {
-        const int slot_i = static_cast<int>(s % kStages);
-        const int use = static_cast<int>(s / kStages);
-        if (use >= 1) {
-          bool ok = true;
-          if (lane == 0) ok = mbar_wait(&empty[slot_i], (use - 1) & 1);
-          ok = __shfl_sync(0xffffffffu, ok, 0);
-          if (!ok || *abort_flag) {
-            if (!ok && lane == 0) set_err(a.err, PKV_DEV_ERR_TIMEOUT);
-            *abort_flag = 1;
-            aborted = true;
-            break;
-          }
+    for (int64_t s = 0; h0; ++s) {
+      const int32_t e2 = lookup(c2, h2);
+      const int slot_i = static_cast<int>(s % kStages);
+      const int use = static_cast<int>(s / kStages);
+      if (use >= 1) {
+        bool ok = true;
+        if (lane == 0) ok = mbar_wait(&empty[slot_i], (use - 1) & 1);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (__any_sync(0xffffffffu, !ok || *abort_flag != 0)) {
+          if (!ok && lane == 0) set_err(a.err, PKV_DEV_ERR_TIMEOUT);
+          *abort_flag = 1;
+          break;
         }
-        uint8_t* kst = ring + slot_i * L.stage_bytes;
-        uint8_t* vst = kst + T * a.row_bytes;
-        const int64_t j = j0 + lane;
-        const bool in_piece = lane < T && j < jb;
-        int64_t slot = -1;
-        if (in_piece && row_ok) slot = token_slot(rowp, j, a.page_size, a.num_slots, a.err);
-        const bool load = in_piece && slot >= 0;
-        if (in_piece && !load) {
-          // Out-of-range entry: the row reads as zeros (error already flagged).
-          for (int b = 0; b < a.row_bytes; b += 16) {
-            *reinterpret_cast<uint4*>(kst + lane * a.row_bytes + b) = make_uint4(0, 0, 0, 0);
-            *reinterpret_cast<uint4*>(vst + lane * a.row_bytes + b) = make_uint4(0, 0, 0, 0);
-          }
-          // Later bulk copies (async proxy) may write these bytes again.
-          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        }
-        const unsigned nload = __popc(__ballot_sync(0xffffffffu, load));
-        __syncwarp();
-        if (lane == 0) mbar_arrive_expect_tx(&full[slot_i], nload * 2u * a.row_bytes);
-        __syncwarp();
-        if (load) {
-          bulk_g2s(kst + lane * a.row_bytes, a.kbase + slot * a.slot_stride_bytes, a.row_bytes,
-                   &full[slot_i], policy);
-          bulk_g2s(vst + lane * a.row_bytes, a.vbase + slot * a.slot_stride_bytes, a.row_bytes,
-                   &full[slot_i], policy);
-        }
-        last_use[slot_i] = use;
       }
+      uint8_t* kst = ring + slot_i * L.stage_bytes;
+      uint8_t* vst = kst + T * a.row_bytes;
+      const int64_t j = c0.j0 + lane;
+      const bool in_piece = lane < T && j < c0.jb;
+      int64_t slot = -1;
+      if (in_piece && c0.row_ok) {
+        bool aligned = true;
+        if (a.page_size == 1) {
+          slot = e0;
+        } else if (e0 % a.page_size == 0) {
+          slot = static_cast<int64_t>(e0 / a.page_size) * a.page_size + (j % a.page_size);
+        } else {
+          aligned = false;
+          set_err(a.err, PKV_DEV_ERR_PAGE_ALIGN);
+        }
+        if (aligned && (slot < 0 || slot >= a.num_slots)) {
+          set_err(a.err, PKV_DEV_ERR_SLOT_RANGE);
+          slot = -1;
+        }
+      }
+      const bool load = in_piece && slot >= 0;
+      if (in_piece && !load) {
+        // Out-of-range entry: the row reads as zeros (error already flagged).
+        for (int b = 0; b < a.row_bytes; b += 16) {
+          *reinterpret_cast<uint4*>(kst + lane * a.row_bytes + b) = make_uint4(0, 0, 0, 0);
+          *reinterpret_cast<uint4*>(vst + lane * a.row_bytes + b) = make_uint4(0, 0, 0, 0);
+        }
+        // Later bulk copies (async proxy) may write these bytes again.
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      }
+      const unsigned nload = __popc(__ballot_sync(0xffffffffu, load));
+      __syncwarp();
+      if (lane == 0) mbar_arrive_expect_tx(&full[slot_i], nload * 2u * a.row_bytes);
+      __syncwarp();
+      if (load) {
+        bulk_g2s(kst + lane * a.row_bytes, a.kbase + slot * a.slot_stride_bytes, a.row_bytes,
+                 &full[slot_i], policy);
+        bulk_g2s(vst + lane * a.row_bytes, a.vbase + slot * a.slot_stride_bytes, a.row_bytes,
+                 &full[slot_i], policy);
+      }
+      last_use[slot_i] = use;
+      // Shift the look-ahead window.
+      c0 = c1;
+      h0 = h1;
+      e0 = e1;
+      c1 = c2;
+      h1 = h2;
+      e1 = e2;
+      if (h2) h2 = advance(c2);
     }
     // Make sure no copy into this CTA's shared memory is still in flight.
     if (lane == 0) {
@@ -463,12 +525,16 @@ __global__ void __launch_bounds__(32 * 9, 1) decode_split_kernel(const DecodeArg
 }
 
 // Merge the pieces of requests that spanned more than one CTA; zero the rows
-// of empty contexts.  One warp per (request, q head); lane owns 4 dims.
+// of empty contexts.  One warp per (request, q head); lane owns 4 dims.  The
+// pieces' (max, sum) pairs are read in parallel across lanes and the partial
+// rows with independent loads, so the merge costs a few memory round trips.
 template <typename E>
 __global__ void __launch_bounds__(128) decode_combine_kernel(
     const int32_t* __restrict__ seq_lens, const int32_t* __restrict__ cum,
     const int64_t* __restrict__ per_p, const float2* __restrict__ ml, const float* __restrict__ o,
     int32_t hq, void* __restrict__ out) {
+  // Partials come from the split kernel launched just before this one.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int r = blockIdx.x;
   const int h = blockIdx.y * 4 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
@@ -487,14 +553,17 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(
   const int64_t k_lo = c0 / per, k_hi = (c1 - 1) / per;
   if (k_lo == k_hi) return;  // written by its only piece
   float M = -INFINITY;
-  for (int64_t k = k_lo; k <= k_hi; ++k) M = fmaxf(M, ml[(k + r) * hq + h].x);
+  for (int64_t k = k_lo + lane; k <= k_hi; k += 32) M = fmaxf(M, ml[(k + r) * hq + h].x);
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
   float4 acc = make_float4(0, 0, 0, 0);
   float den = 0.f;
+#pragma unroll 4
   for (int64_t k = k_lo; k <= k_hi; ++k) {
     const float2 st = ml[(k + r) * hq + h];
+    const float4 x = *reinterpret_cast<const float4*>(o + ((k + r) * hq + h) * kHeadDim + 4 * lane);
     const float w = exp2f(st.x - M);
     den += w * st.y;
-    const float4 x = *reinterpret_cast<const float4*>(o + ((k + r) * hq + h) * kHeadDim + 4 * lane);
     acc.x += w * x.x;
     acc.y += w * x.y;
     acc.z += w * x.z;
@@ -518,13 +587,30 @@ cudaError_t launch_decode_t(const DecodeArgs& a, int grid, cudaStream_t s) {
   cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<E, G>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, L.total);
   if (e != cudaSuccess) return e;
-  decode_split_kernel<E, G><<<grid, 32 * (1 + a.hkv), L.total, s>>>(a);
-  e = cudaGetLastError();
+  // Both kernels use programmatic dependent launch: the split kernel's set-up
+  // (barriers, length scan, first table reads) overlaps the tail of the
+  // preceding kernel and waits (griddepcontrol.wait) before reading the pool;
+  // the combine kernel is scheduled while the split kernel runs and waits
+  // for its partials.
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(32 * (1 + a.hkv));
+  cfg.dynamicSmemBytes = L.total;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, decode_split_kernel<E, G>, a);
   if (e != cudaSuccess) return e;
-  dim3 cg(a.batch, (a.hq + 3) / 4);
-  decode_combine_kernel<E><<<cg, 128, 0, s>>>(a.seq_lens, a.ws_cum, a.ws_per, a.ws_ml, a.ws_o,
-                                              a.hq, a.out);
-  return cudaGetLastError();
+  cudaLaunchConfig_t ccfg = cfg;
+  ccfg.gridDim = dim3(a.batch, (a.hq + 3) / 4);
+  ccfg.blockDim = dim3(128);
+  ccfg.dynamicSmemBytes = 0;
+  return cudaLaunchKernelEx(&ccfg, decode_combine_kernel<E>, a.seq_lens, (const int32_t*)a.ws_cum,
+                            (const int64_t*)a.ws_per, (const float2*)a.ws_ml, (const float*)a.ws_o,
+                            a.hq, a.out);
 }
 
 }  // namespace

@@ -9,23 +9,27 @@
 // sits at position prefix + i and sees keys 0 .. prefix + i; query head h
 // reads KV head h / (Hq/Hkv).
 //
-// Design (B200, one CTA per SM, 12 warps):
+// Design (B200, one CTA per SM, 13 warps):
 //  * A CTA owns one (request, KV head, 2 x 128 query rows) block.  Rows are
 //    (token, query head of the group) pairs, token-major, so the G query heads
 //    sharing a KV head form the M dimension of one MMA and every K/V tile is
 //    used by 256 rows.
-//  * warp 0 -- loads: the two Q tiles once (3-D TMA boxes [tokens][G heads][64
-//    dims] with the 128-byte swizzle), then for each 128-key tile it
-//    translates the keys' slots through the page table and gathers the K and V
-//    rows with TMA tile::gather4 (4 pool rows per copy, 128-byte swizzle) into
-//    a 2-stage ring.  The gathered layout is directly the UMMA operand layout:
-//    K-major for K (B of Q K^T), MN-major for V (B of P V).
-//  * warp 1 -- MMA issue (one thread): S_i = Q_i K^T into TMEM (M=128, N=128,
-//    K=16 steps), then O_i += P_i V with P_i read from TMEM.  Issue order
-//    PV_0(j), QK_0(j+1), PV_1(j), QK_1(j+1) lets softmax of one Q tile run
-//    while the tensor core works on the other.  Completion is signalled with
-//    tcgen05.commit to mbarriers.  The warp also allocates / frees TMEM.
-//  * warps 4-7 and 8-11 -- softmax for Q tile 0 and 1: one thread per row,
+//  * warps 8-11 -- K/V loads: two groups of two warps, each owning one stage
+//    of a 2-deep ring.  For each 128-key tile a group translates the keys'
+//    slots through the page table (one tile ahead) and moves the 256-byte head
+//    rows with 16-byte cp.async copies straight into the 128-byte-swizzled
+//    UMMA operand layout: K-major for K (B of Q K^T), MN-major for V (B of
+//    P V).  A lane pair of half-warps covers two rows per step, so every warp
+//    access is two fully used 256-byte segments.  (TMA tile::gather4 was tried
+//    first: four 128-byte rows per instruction issued too slowly to feed the
+//    tensor core.)
+//  * warp 12 -- the two Q tiles by 3-D TMA boxes [tokens][G heads][64 dims]
+//    (128-byte swizzle), TMEM allocation, and MMA issue (one thread):
+//    S_i = Q_i K^T into TMEM (M=128, N=128, K=16 steps), then O_i += P_i V with
+//    P_i read from TMEM.  Issue order PV_0(j), QK_0(j+1), PV_1(j), QK_1(j+1)
+//    lets softmax of one Q tile run while the tensor core works on the other.
+//    Completion is signalled with tcgen05.commit to mbarriers.
+//  * warps 0-3 and 4-7 -- softmax for Q tile 0 and 1: one thread per row,
 //    tcgen05.ld of its S row, log2-domain online softmax with a lazily moved
 //    max (O rescaled in TMEM only when the max grows by more than 2^8), P
 //    written back over S as packed bf16 with tcgen05.st; at the end O / l is
@@ -52,7 +56,10 @@ constexpr int kQTiles = 2;
 constexpr int kKvStages = 2;
 constexpr int kHalfBytes = 128 * 128;     // 128 rows x 64 bf16 (one swizzle column block)
 constexpr int kTileBytes = 2 * kHalfBytes;  // 128 rows x 128 bf16
-constexpr int kThreads = 384;
+constexpr int kThreads = 416;  // 13 warps
+constexpr int kWarpMma = 12;    // MMA issue, Q load, TMEM allocation
+constexpr int kWarpLoad0 = 8;   // warps 8-11: K/V gathers (two groups of two warps)
+constexpr int kLoadThreadsPerGroup = 64;
 
 // Shared memory map (offsets from a 1024-byte aligned base).
 constexpr int kOffQ = 0;
@@ -82,6 +89,9 @@ constexpr uint32_t kColO = 256;  // + 128 * tile
 constexpr float kRescaleThreshold = 8.0f;
 
 struct ExtendTcArgs {
+  const uint8_t* kbase;  // layer base of the K plane (bytes)
+  const uint8_t* vbase;
+  int64_t slot_stride_bytes;
   const int32_t* table;
   int64_t table_rows, table_cols, table_stride;
   int32_t page_size;
@@ -105,16 +115,6 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, i
       "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar))
-      : "memory");
-}
-
-__device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* map, int col, int r0, int r1,
-                                            int r2, int r3, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(col), "r"(r0), "r"(r1), "r"(r2), "r"(r3),
-      "r"(smem_u32(bar))
       : "memory");
 }
 
@@ -216,11 +216,24 @@ __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+// 2^x on the SFU (approximate, flushes subnormal results to zero).
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Three-input maximum (one instruction on sm_100).
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 // ---- the kernel ---------------------------------------------------------------
 template <int G>
 __global__ void __launch_bounds__(kThreads, 1)
-    extend_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
-                     const __grid_constant__ CUtensorMap vmap, const ExtendTcArgs a) {
+    extend_tc_kernel(const __grid_constant__ CUtensorMap qmap, const ExtendTcArgs a) {
   constexpr int TQ = kRowsPerTile / G;  // tokens per Q tile
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -257,9 +270,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     mbar_init(&bars[kBarQFull], 1);
     for (int s = 0; s < kKvStages; ++s) {
-      mbar_init(&bars[kBarKFull + s], 1);
+      mbar_init(&bars[kBarKFull + s], kLoadThreadsPerGroup);
       mbar_init(&bars[kBarKEmpty + s], 1);
-      mbar_init(&bars[kBarVFull + s], 1);
+      mbar_init(&bars[kBarVFull + s], kLoadThreadsPerGroup);
       mbar_init(&bars[kBarVEmpty + s], 1);
     }
     for (int i = 0; i < kQTiles; ++i) {
@@ -271,7 +284,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 1) {
+  if (warp == kWarpMma) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
                  "r"(kTmemCols)
                  : "memory");
@@ -286,79 +299,93 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sK = smem + kOffK;
   uint8_t* sV = smem + kOffV;
 
-  if (warp == 0) {
-    // ============================ loads =======================================
+  if (warp >= kWarpLoad0 && warp < kWarpMma) {
+    // ============================ K/V gathers =================================
+    // Two groups of two warps; group grp owns ring stage grp and loads tiles
+    // grp, grp + 2, ...  A warp copies 64 keys of the tile: in each step lanes
+    // 0-15 and 16-31 move the 256-byte head rows of two keys as 16-byte
+    // cp.async chunks, written at their 128-byte-swizzle positions (chunk c of
+    // key k goes to column block c/8, row k, 16-byte slot (c%8) ^ (k%8)), which
+    // is the UMMA operand layout.  Each group waits for its own copies, makes
+    // them visible to the tensor core (fence.proxy.async) and arrives on the
+    // stage's full barrier: K first, then V.
+    const int grp = (warp - kWarpLoad0) >> 1;
+    const int gw = (warp - kWarpLoad0) & 1;
+    const int h = lane >> 4, c = lane & 15;
     const int32_t* rowp = a.table + (row_ok ? trow : 0) * a.table_stride;
-    if (lane == 0) {
-      mbar_arrive_expect_tx(&bars[kBarQFull], kQTiles * kTileBytes);
-      for (int i = 0; i < kQTiles; ++i)
-        for (int h = 0; h < 2; ++h)
-          tma_load_3d(sQ + i * kTileBytes + h * kHalfBytes, &qmap, h * 64, g * G,
-                      static_cast<int>(qbase + i0 + i * TQ), &bars[kBarQFull]);
-    }
     // A masked key reads the request's first key row (finite, part of its context).
     int32_t dummy = 0;
     if (row_ok) {
       const int64_t s0 = token_slot(rowp, 0, a.page_size, a.num_slots, nullptr);
       dummy = s0 >= 0 ? static_cast<int32_t>(s0) : 0;
     }
-    int k_last_use[kKvStages] = {-1, -1};
-    int v_last_use[kKvStages] = {-1, -1};
-    bool ok = true;
-    for (int j = 0; j < ntiles && ok; ++j) {
-      const int st = j & 1, use = j >> 1;
-      int rows[4];
+    // Slots of keys gw*64 + lane and gw*64 + 32 + lane of tile jj.
+    auto lookup = [&](int jj, int32_t (&sl)[2]) {
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int64_t key = static_cast<int64_t>(j) * kKeysPerTile + lane * 4 + u;
-        int64_t s = -1;
-        if (key < kv_end && row_ok) s = token_slot(rowp, key, a.page_size, a.num_slots, a.err);
-        rows[u] = s >= 0 ? static_cast<int32_t>(s) : dummy;
+      for (int u = 0; u < 2; ++u) {
+        const int64_t key = static_cast<int64_t>(jj) * kKeysPerTile + gw * 64 + u * 32 + lane;
+        int64_t sv = -1;
+        if (jj < ntiles && key < kv_end && row_ok) sv = token_slot(rowp, key, a.page_size, a.num_slots, a.err);
+        sl[u] = sv >= 0 ? static_cast<int32_t>(sv) : dummy;
       }
+    };
+    auto copy_tile = [&](const uint8_t* base, uint32_t dst_tile, const int32_t (&sl)[2]) {
+#pragma unroll 8
+      for (int t = 0; t < 32; ++t) {
+        const int kl = 2 * t + h;  // key within this warp's 64
+        const int32_t slot = __shfl_sync(0xffffffffu, kl < 32 ? sl[0] : sl[1], kl & 31);
+        const int kk = gw * 64 + kl;  // key within the tile
+        const uint8_t* src = base + static_cast<int64_t>(slot) * a.slot_stride_bytes + g * 256 + c * 16;
+        const uint32_t dst = dst_tile + (c >> 3) * kHalfBytes + kk * 128 + (((c & 7) ^ (kk & 7)) << 4);
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+      }
+      asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+    const uint32_t k_dst = smem_u32(sK + grp * kTileBytes);
+    const uint32_t v_dst = smem_u32(sV + grp * kTileBytes);
+    int32_t sl[2];
+    lookup(grp, sl);
+    for (int j = grp; j < ntiles; j += 2) {
+      const int use = j >> 1;
       if (use >= 1) {
-        bool w = true;
-        if (lane == 0) w = mbar_wait(&bars[kBarKEmpty + st], (use - 1) & 1);
-        w = __shfl_sync(0xffffffffu, w, 0);
-        if (__any_sync(0xffffffffu, !w || *abort_flag != 0)) { ok = false; break; }
+        const bool w = mbar_wait(&bars[kBarKEmpty + grp], (use - 1) & 1);
+        if (__any_sync(0xffffffffu, !w || *abort_flag != 0)) {
+          if (lane == 0 && !w) set_err(a.err, PKV_DEV_ERR_TIMEOUT);
+          *abort_flag = 1;
+          break;
+        }
       }
-      if (lane == 0) mbar_arrive_expect_tx(&bars[kBarKFull + st], kTileBytes);
-      __syncwarp();
-#pragma unroll
-      for (int h = 0; h < 2; ++h)
-        tma_gather4(sK + st * kTileBytes + h * kHalfBytes + lane * 4 * 128, &kmap, g * 128 + h * 64,
-                    rows[0], rows[1], rows[2], rows[3], &bars[kBarKFull + st]);
-      k_last_use[st] = use;
+      copy_tile(a.kbase, k_dst, sl);
+      asm volatile("cp.async.wait_group 0;" ::: "memory");
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      mbar_arrive(&bars[kBarKFull + grp]);
       if (use >= 1) {
-        bool w = true;
-        if (lane == 0) w = mbar_wait(&bars[kBarVEmpty + st], (use - 1) & 1);
-        w = __shfl_sync(0xffffffffu, w, 0);
-        if (__any_sync(0xffffffffu, !w || *abort_flag != 0)) { ok = false; break; }
+        const bool w = mbar_wait(&bars[kBarVEmpty + grp], (use - 1) & 1);
+        if (__any_sync(0xffffffffu, !w || *abort_flag != 0)) {
+          if (lane == 0 && !w) set_err(a.err, PKV_DEV_ERR_TIMEOUT);
+          *abort_flag = 1;
+          break;
+        }
       }
-      if (lane == 0) mbar_arrive_expect_tx(&bars[kBarVFull + st], kTileBytes);
-      __syncwarp();
-#pragma unroll
-      for (int h = 0; h < 2; ++h)
-        tma_gather4(sV + st * kTileBytes + h * kHalfBytes + lane * 4 * 128, &vmap, g * 128 + h * 64,
-                    rows[0], rows[1], rows[2], rows[3], &bars[kBarVFull + st]);
-      v_last_use[st] = use;
+      copy_tile(a.vbase, v_dst, sl);
+      int32_t nsl[2];
+      lookup(j + 2, nsl);  // next tile's slots load while these copies fly
+      asm volatile("cp.async.wait_group 0;" ::: "memory");
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      mbar_arrive(&bars[kBarVFull + grp]);
+      sl[0] = nsl[0];
+      sl[1] = nsl[1];
     }
-    if (!ok && lane == 0) {
-      set_err(a.err, PKV_DEV_ERR_TIMEOUT);
-      *abort_flag = 1;
-    }
-    // Every copy issued into this CTA's shared memory must land before exit.
+    // No copy into this CTA's shared memory may outlive the loop.
+    asm volatile("cp.async.wait_all;" ::: "memory");
+  } else if (warp == kWarpMma) {
+    // ============================ Q load + MMA issue ==========================
     if (lane == 0) {
-      if (!mbar_wait(&bars[kBarQFull], 0)) set_err(a.err, PKV_DEV_ERR_TIMEOUT);
-      for (int s = 0; s < kKvStages; ++s) {
-        if (k_last_use[s] >= 0 && !mbar_wait(&bars[kBarKFull + s], k_last_use[s] & 1))
-          set_err(a.err, PKV_DEV_ERR_TIMEOUT);
-        if (v_last_use[s] >= 0 && !mbar_wait(&bars[kBarVFull + s], v_last_use[s] & 1))
-          set_err(a.err, PKV_DEV_ERR_TIMEOUT);
-      }
-    }
-  } else if (warp == 1) {
-    // ============================ MMA issue ===================================
-    if (lane == 0) {
+      mbar_arrive_expect_tx(&bars[kBarQFull], kQTiles * kTileBytes);
+      for (int i = 0; i < kQTiles; ++i)
+        for (int h = 0; h < 2; ++h)
+          tma_load_3d(sQ + i * kTileBytes + h * kHalfBytes, &qmap, h * 64, g * G,
+                      static_cast<int>(qbase + i0 + i * TQ), &bars[kBarQFull]);
       const uint32_t q_addr = smem_u32(sQ);
       const uint32_t k_addr = smem_u32(sK);
       const uint32_t v_addr = smem_u32(sV);
@@ -425,9 +452,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!mbar_wait(&bars[kBarOFinal], 0)) set_err(a.err, PKV_DEV_ERR_TIMEOUT);
     }
     __syncwarp();
-  } else if (warp >= 4) {
+  } else if (warp < kWarpLoad0) {
     // ============================ softmax + epilogue ==========================
-    const int i = (warp - 4) >> 2;   // Q tile
+    const int i = warp >> 2;         // Q tile
     const int wq = warp & 3;         // TMEM lane quadrant
     const int m = wq * 32 + lane;    // row within the tile
     const int tq = m / G, hh = m % G;
@@ -437,30 +464,39 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
     const uint32_t s_addr = tmem + lane_base + kColS + 128 * i;
     const uint32_t o_addr = tmem + lane_base + kColO + 128 * i;
-    float m_run = -INFINITY, l_run = 0.f;
+    float m_run = -INFINITY;
+    float2 l2 = make_float2(0.f, 0.f);  // running sum of p, even / odd keys
+    const float2 sl2 = make_float2(a.scale_log2, a.scale_log2);
     bool ok = true;
     for (int j = 0; j < ntiles; ++j) {
       const bool w = mbar_wait(&bars[kBarSFull + i], j & 1);
       if (__any_sync(0xffffffffu, !w || *abort_flag != 0)) { ok = false; break; }
       tc_fence_after();
       const int64_t kb = static_cast<int64_t>(j) * kKeysPerTile;
-      const bool full_tile = kb + kKeysPerTile <= lim;
+      // Keys kb .. kb + vis - 1 of this tile are visible to this row.
+      const int64_t vis64 = lim - kb;
+      const int32_t vis = vis64 <= 0 ? 0 : (vis64 >= kKeysPerTile ? kKeysPerTile : static_cast<int32_t>(vis64));
+      const bool warp_full = __all_sync(0xffffffffu, vis == kKeysPerTile);
+      // ---- pass 1: row max of the raw scores ----
       float mx = -INFINITY;
 #pragma unroll 1
       for (int c = 0; c < 4; ++c) {
         float v[32];
         tmem_ld32(s_addr + c * 32, v);
+        if (warp_full) {
 #pragma unroll
-        for (int u = 0; u < 32; ++u) {
-          const bool vis = full_tile || (kb + c * 32 + u < lim);
-          mx = vis ? fmaxf(mx, v[u]) : mx;
+          for (int u = 0; u < 32; u += 2) mx = max3f(mx, v[u], v[u + 1]);
+        } else {
+#pragma unroll
+          for (int u = 0; u < 32; ++u) mx = (c * 32 + u < vis) ? fmaxf(mx, v[u]) : mx;
         }
       }
       mx *= a.scale_log2;
       const bool need = mx > m_run + kRescaleThreshold;
       if (j > 0 && __any_sync(0xffffffffu, need)) {
-        const float alpha = need ? exp2f(m_run - mx) : 1.f;
-        l_run *= alpha;
+        const float alpha = need ? ex2_approx(m_run - mx) : 1.f;
+        l2.x *= alpha;
+        l2.y *= alpha;
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
           float o[32];
@@ -472,20 +508,30 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait_st();
       }
       if (need) m_run = mx;
-      const float neg_m = -m_run;
+      const float2 negm2 = make_float2(-m_run, -m_run);
+      // ---- pass 2: p = 2^(s * scale * log2e - m), packed to bf16 over S ----
 #pragma unroll 1
       for (int c = 0; c < 4; ++c) {
         float v[32];
         tmem_ld32(s_addr + c * 32, v);
         uint32_t w16[16];
+        if (warp_full) {
 #pragma unroll
-        for (int u = 0; u < 32; u += 2) {
-          const bool vis0 = full_tile || (kb + c * 32 + u < lim);
-          const bool vis1 = full_tile || (kb + c * 32 + u + 1 < lim);
-          const float p0 = vis0 ? exp2f(fmaf(v[u], a.scale_log2, neg_m)) : 0.f;
-          const float p1 = vis1 ? exp2f(fmaf(v[u + 1], a.scale_log2, neg_m)) : 0.f;
-          l_run += p0 + p1;
-          w16[u >> 1] = pack_bf16x2(p0, p1);
+          for (int u = 0; u < 32; u += 2) {
+            const float2 t = __ffma2_rn(make_float2(v[u], v[u + 1]), sl2, negm2);
+            const float2 pp = make_float2(ex2_approx(t.x), ex2_approx(t.y));
+            l2 = __fadd2_rn(l2, pp);
+            w16[u >> 1] = pack_bf16x2(pp.x, pp.y);
+          }
+        } else {
+#pragma unroll
+          for (int u = 0; u < 32; u += 2) {
+            const float2 t = __ffma2_rn(make_float2(v[u], v[u + 1]), sl2, negm2);
+            const float p0 = (c * 32 + u < vis) ? ex2_approx(t.x) : 0.f;
+            const float p1 = (c * 32 + u + 1 < vis) ? ex2_approx(t.y) : 0.f;
+            l2 = __fadd2_rn(l2, make_float2(p0, p1));
+            w16[u >> 1] = pack_bf16x2(p0, p1);
+          }
         }
         tmem_st16(s_addr + c * 16, w16);
       }
@@ -493,6 +539,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(&bars[kBarPReady + i]);
     }
+    const float l_run = l2.x + l2.y;
     if (!ok && lane == 0) {
       set_err(a.err, PKV_DEV_ERR_TIMEOUT);
       *abort_flag = 1;
@@ -528,7 +575,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 1) {
+  if (warp == kWarpMma) {
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols)
                  : "memory");
   }
@@ -547,18 +594,6 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-bool make_row_map(CUtensorMap* map, const void* base, int64_t row_elems, int64_t rows, int64_t row_stride_bytes) {
-  auto fn = encode_fn();
-  if (fn == nullptr) return false;
-  cuuint64_t dims[2] = {static_cast<cuuint64_t>(row_elems), static_cast<cuuint64_t>(rows)};
-  cuuint64_t strides[1] = {static_cast<cuuint64_t>(row_stride_bytes)};
-  cuuint32_t box[2] = {64, 1};
-  cuuint32_t estr[2] = {1, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 bool make_q_map(CUtensorMap* map, const void* q, int32_t hq, int64_t total_q, int G) {
   auto fn = encode_fn();
   if (fn == nullptr) return false;
@@ -572,14 +607,14 @@ bool make_q_map(CUtensorMap* map, const void* q, int32_t hq, int64_t total_q, in
 }
 
 template <int G>
-cudaError_t launch_g(const CUtensorMap& qm, const CUtensorMap& km, const CUtensorMap& vm, const ExtendTcArgs& a,
+cudaError_t launch_g(const CUtensorMap& qm, const ExtendTcArgs& a,
                      int32_t batch, int32_t max_extend, cudaStream_t s) {
   constexpr int TQ = kRowsPerTile / G;
   const int nqb = (max_extend + kQTiles * TQ - 1) / (kQTiles * TQ);
   cudaError_t e = cudaFuncSetAttribute(extend_tc_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
   dim3 grid(nqb, a.hkv, batch);
-  extend_tc_kernel<G><<<grid, kThreads, kSmemBytes, s>>>(qm, km, vm, a);
+  extend_tc_kernel<G><<<grid, kThreads, kSmemBytes, s>>>(qm, a);
   return cudaGetLastError();
 }
 
@@ -591,13 +626,12 @@ cudaError_t launch_extend_tc(const PoolView& pool, const TableView& t, const voi
                              float scale, void* out, int32_t* err, cudaStream_t s) {
   if (batch == 0 || max_extend == 0 || total_q == 0) return cudaSuccess;
   const int G = num_q_heads / pool.num_kv_heads;
-  CUtensorMap qm, km, vm;
-  const int64_t row_elems = static_cast<int64_t>(pool.num_kv_heads) * kHeadDimHost;
-  if (!make_q_map(&qm, q, num_q_heads, total_q, G) ||
-      !make_row_map(&km, pool.k, row_elems, pool.num_slots, pool.slot_stride_bytes) ||
-      !make_row_map(&vm, pool.v, row_elems, pool.num_slots, pool.slot_stride_bytes))
-    return cudaErrorInvalidValue;
+  CUtensorMap qm;
+  if (!make_q_map(&qm, q, num_q_heads, total_q, G)) return cudaErrorInvalidValue;
   ExtendTcArgs a;
+  a.kbase = pool.k;
+  a.vbase = pool.v;
+  a.slot_stride_bytes = pool.slot_stride_bytes;
   a.table = t.entries;
   a.table_rows = t.rows;
   a.table_cols = t.cols;
@@ -616,10 +650,10 @@ cudaError_t launch_extend_tc(const PoolView& pool, const TableView& t, const voi
   a.scale_log2 = scale * kLog2e;
   a.err = err;
   switch (G) {
-    case 1: return launch_g<1>(qm, km, vm, a, batch, max_extend, s);
-    case 2: return launch_g<2>(qm, km, vm, a, batch, max_extend, s);
-    case 4: return launch_g<4>(qm, km, vm, a, batch, max_extend, s);
-    case 8: return launch_g<8>(qm, km, vm, a, batch, max_extend, s);
+    case 1: return launch_g<1>(qm, a, batch, max_extend, s);
+    case 2: return launch_g<2>(qm, a, batch, max_extend, s);
+    case 4: return launch_g<4>(qm, a, batch, max_extend, s);
+    case 8: return launch_g<8>(qm, a, batch, max_extend, s);
   }
   return cudaErrorInvalidValue;
 }

@@ -19,6 +19,9 @@ __global__ void __launch_bounds__(256) store_kv_kernel(
     int64_t num_slots, const uint8_t* __restrict__ k, int64_t k_stride_bytes,
     const uint8_t* __restrict__ v, int64_t v_stride_bytes, const void* __restrict__ out_loc,
     int loc_i64, int64_t n, int32_t chunks_per_row, int32_t* err) {
+  // The attention kernel that follows may start its set-up now; it waits for
+  // this grid before it reads the pool.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int64_t total = n * 2 * chunks_per_row;
   for (int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; idx < total;
        idx += (int64_t)gridDim.x * blockDim.x) {
