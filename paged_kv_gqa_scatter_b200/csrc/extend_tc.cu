@@ -9,13 +9,13 @@
 // sits at position prefix + i and sees keys 0 .. prefix + i; query head h
 // reads KV head h / (Hq/Hkv).
 //
-// Design (B200, one CTA per SM, 13 warps):
+// Design (B200, one CTA per SM, 11 warps):
 //  * A CTA owns one (request, KV head, 2 x 128 query rows) block.  Rows are
 //    (token, query head of the group) pairs, token-major, so the G query heads
 //    sharing a KV head form the M dimension of one MMA and every K/V tile is
 //    used by 256 rows.
-//  * warps 8-11 -- K/V loads: two groups of two warps, each owning one stage
-//    of a 2-deep ring.  For each 128-key tile a group translates the keys'
+//  * warps 8 and 9 -- K/V loads: each warp owns one stage of a 2-deep ring
+//    and loads every other tile.  For each 128-key tile a warp translates the keys'
 //    slots through the page table (one tile ahead) and moves the 256-byte head
 //    rows with 16-byte cp.async copies straight into the 128-byte-swizzled
 //    UMMA operand layout: K-major for K (B of Q K^T), MN-major for V (B of
@@ -23,14 +23,14 @@
 //    access is two fully used 256-byte segments.  (TMA tile::gather4 was tried
 //    first: four 128-byte rows per instruction issued too slowly to feed the
 //    tensor core.)
-//  * warp 12 -- the two Q tiles by 3-D TMA boxes [tokens][G heads][64 dims]
+//  * warp 10 -- the two Q tiles by 3-D TMA boxes [tokens][G heads][64 dims]
 //    (128-byte swizzle), TMEM allocation, and MMA issue (one thread):
 //    S_i = Q_i K^T into TMEM (M=128, N=128, K=16 steps), then O_i += P_i V with
 //    P_i read from TMEM.  Issue order PV_0(j), QK_0(j+1), PV_1(j), QK_1(j+1)
 //    lets softmax of one Q tile run while the tensor core works on the other.
 //    Completion is signalled with tcgen05.commit to mbarriers.
 //  * warps 0-3 and 4-7 -- softmax for Q tile 0 and 1: one thread per row,
-//    tcgen05.ld of its S row, log2-domain online softmax with a lazily moved
+//    the S row read from TMEM in one go, log2-domain online softmax with a lazily moved
 //    max (O rescaled in TMEM only when the max grows by more than 2^8), P
 //    written back over S as packed bf16 with tcgen05.st; at the end O / l is
 //    read from TMEM and stored as bf16.
@@ -51,39 +51,42 @@ namespace pkv {
 namespace {
 
 constexpr int kRowsPerTile = 128;
-constexpr int kKeysPerTile = 128;
+constexpr int kKeysPerStep = 64;                  // keys per softmax step / K,V ring stage
 constexpr int kQTiles = 2;
-constexpr int kKvStages = 2;
-constexpr int kHalfBytes = 128 * 128;     // 128 rows x 64 bf16 (one swizzle column block)
-constexpr int kTileBytes = 2 * kHalfBytes;  // 128 rows x 128 bf16
-constexpr int kThreads = 416;  // 13 warps
-constexpr int kWarpMma = 12;    // MMA issue, Q load, TMEM allocation
-constexpr int kWarpLoad0 = 8;   // warps 8-11: K/V gathers (two groups of two warps)
-constexpr int kLoadThreadsPerGroup = 64;
+constexpr int kKvStages = 4;
+constexpr int kQHalfBytes = 128 * 128;            // 128 rows x 64 bf16 (one 128-byte column block)
+constexpr int kQTileBytes = 2 * kQHalfBytes;      // 128 rows x 128 bf16
+constexpr int kKvHalfBytes = kKeysPerStep * 128;  // 64 keys x 64 bf16
+constexpr int kKvTileBytes = 2 * kKvHalfBytes;    // 64 keys x 128 bf16
+constexpr int kThreads = 352;  // 11 warps
+constexpr int kWarpLoad0 = 8;   // warps 8 and 9: K/V gathers (even / odd steps)
+constexpr int kWarpMma = 10;    // MMA issue, Q load, TMEM allocation
+constexpr int kLoadThreads = 32;
 
 // Shared memory map (offsets from a 1024-byte aligned base).
 constexpr int kOffQ = 0;
-constexpr int kOffK = kOffQ + kQTiles * kTileBytes;
-constexpr int kOffV = kOffK + kKvStages * kTileBytes;
-constexpr int kOffBar = kOffV + kKvStages * kTileBytes;
-constexpr int kNumBars = 16;
+constexpr int kOffK = kOffQ + kQTiles * kQTileBytes;
+constexpr int kOffV = kOffK + kKvStages * kKvTileBytes;
+constexpr int kOffBar = kOffV + kKvStages * kKvTileBytes;
+constexpr int kNumBars = 32;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;
 constexpr int kSmemBytes = kOffMisc + 64 + 1024;  // + slack for manual 1024-byte alignment
 
-// Barrier indices.
+// Barrier indices.  Barriers touched once per step come in pairs indexed by
+// the step's parity (S half), so none can run two phases ahead of its waiter.
 constexpr int kBarQFull = 0;
-constexpr int kBarKFull = 1;    // +stage
-constexpr int kBarKEmpty = 3;   // +stage
-constexpr int kBarVFull = 5;    // +stage
-constexpr int kBarVEmpty = 7;   // +stage
-constexpr int kBarSFull = 9;    // +q tile
-constexpr int kBarPReady = 11;  // +q tile
-constexpr int kBarOFinal = 13;
-constexpr int kBarDrain = 14;
+constexpr int kBarKFull = 1;    // + stage (4)
+constexpr int kBarKEmpty = 5;   // + stage
+constexpr int kBarVFull = 9;    // + stage
+constexpr int kBarVEmpty = 13;  // + stage
+constexpr int kBarSFull = 17;   // + 2 * q tile + half
+constexpr int kBarPReady = 21;  // + 2 * q tile + half
+constexpr int kBarODone = 25;   // + q tile
+constexpr int kBarOFinal = 27;
 
-// TMEM columns.
+// TMEM columns: S_i (two 64-column halves, one per step parity) and O_i.
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS = 0;    // + 128 * tile
+constexpr uint32_t kColS = 0;    // + 128 * tile + 64 * half
 constexpr uint32_t kColO = 256;  // + 128 * tile
 
 constexpr float kRescaleThreshold = 8.0f;
@@ -136,10 +139,10 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint3
   return d;
 }
 
-// Instruction descriptor, kind::f16: bf16 A/B, fp32 D, M = 128, N = 128.
-constexpr uint32_t kIdescBase = (1u << 4) | (1u << 7) | (1u << 10) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
-constexpr uint32_t kIdescQK = kIdescBase;              // A K-major, B K-major
-constexpr uint32_t kIdescPV = kIdescBase | (1u << 16);  // B (V) MN-major
+// Instruction descriptors, kind::f16: bf16 A/B, fp32 D, M = 128.
+constexpr uint32_t kIdescF16 = (1u << 4) | (1u << 7) | (1u << 10) | ((128u >> 4) << 24);
+constexpr uint32_t kIdescQK = kIdescF16 | ((64u >> 3) << 17);                // N = 64 keys, A and B K-major
+constexpr uint32_t kIdescPV = kIdescF16 | ((128u >> 3) << 17) | (1u << 16);  // N = 128 dims, B (V) MN-major
 
 __device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                        uint32_t accum) {
@@ -182,6 +185,18 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Load 64 consecutive 32-bit TMEM columns of this thread's lane (no wait).
+__device__ __forceinline__ void tmem_ld64_nowait(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x64.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, %48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63}, [%64];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]), "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]), "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
+      : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_wait_ld() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
@@ -230,6 +245,17 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
   return d;
 }
 
+// One lane of the (fully active) warp: true in exactly one lane.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "elect.sync _|p, 0xffffffff;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(pred));
+  return pred != 0;
+}
+
 // ---- the kernel ---------------------------------------------------------------
 template <int G>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -264,23 +290,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     kv_end = a.table_cols;
   }
   if (!row_ok && threadIdx.x == 0) set_err(a.err, PKV_DEV_ERR_TABLE_RANGE);
-  const int ntiles = static_cast<int>((kv_end + kKeysPerTile - 1) / kKeysPerTile);
+  const int nsteps = static_cast<int>((kv_end + kKeysPerStep - 1) / kKeysPerStep);
 
   // ---- setup: barriers and TMEM ------------------------------------------------
   if (threadIdx.x == 0) {
     mbar_init(&bars[kBarQFull], 1);
-    for (int s = 0; s < kKvStages; ++s) {
-      mbar_init(&bars[kBarKFull + s], kLoadThreadsPerGroup);
-      mbar_init(&bars[kBarKEmpty + s], 1);
-      mbar_init(&bars[kBarVFull + s], kLoadThreadsPerGroup);
-      mbar_init(&bars[kBarVEmpty + s], 1);
+    for (int st = 0; st < kKvStages; ++st) {
+      mbar_init(&bars[kBarKFull + st], kLoadThreads);
+      mbar_init(&bars[kBarKEmpty + st], 1);
+      mbar_init(&bars[kBarVFull + st], kLoadThreads);
+      mbar_init(&bars[kBarVEmpty + st], 1);
     }
-    for (int i = 0; i < kQTiles; ++i) {
-      mbar_init(&bars[kBarSFull + i], 1);
-      mbar_init(&bars[kBarPReady + i], 128);
+    for (int b = 0; b < 2 * kQTiles; ++b) {
+      mbar_init(&bars[kBarSFull + b], 1);
+      mbar_init(&bars[kBarPReady + b], 128);
     }
+    for (int i = 0; i < kQTiles; ++i) mbar_init(&bars[kBarODone + i], 1);
     mbar_init(&bars[kBarOFinal], 1);
-    mbar_init(&bars[kBarDrain], 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -301,16 +327,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp >= kWarpLoad0 && warp < kWarpMma) {
     // ============================ K/V gathers =================================
-    // Two groups of two warps; group grp owns ring stage grp and loads tiles
-    // grp, grp + 2, ...  A warp copies 64 keys of the tile: in each step lanes
-    // 0-15 and 16-31 move the 256-byte head rows of two keys as 16-byte
-    // cp.async chunks, written at their 128-byte-swizzle positions (chunk c of
-    // key k goes to column block c/8, row k, 16-byte slot (c%8) ^ (k%8)), which
-    // is the UMMA operand layout.  Each group waits for its own copies, makes
-    // them visible to the tensor core (fence.proxy.async) and arrives on the
-    // stage's full barrier: K first, then V.
-    const int grp = (warp - kWarpLoad0) >> 1;
-    const int gw = (warp - kWarpLoad0) & 1;
+    // Warp par loads steps par, par + 2, ... into ring stages (step % 4).  For
+    // each 64-key step it translates the keys' slots through the page table
+    // (one step ahead) and moves their 256-byte head rows as 16-byte cp.async
+    // chunks: in each instruction lanes 0-15 and 16-31 cover the rows of two
+    // keys, so a warp access is two fully used 256-byte segments.  Chunk c of
+    // key k lands at column block c/8, row k, 16-byte slot (c%8) ^ (k%8): the
+    // 128-byte-swizzled UMMA operand layout (K-major for K, MN-major for V).
+    // K and V copies of a step are in flight together; the warp waits for
+    // each group in turn, makes it visible to the tensor core
+    // (fence.proxy.async) and arrives on the stage's full barrier, K first.
+    const int par = warp - kWarpLoad0;
     const int h = lane >> 4, c = lane & 15;
     const int32_t* rowp = a.table + (row_ok ? trow : 0) * a.table_stride;
     // A masked key reads the request's first key row (finite, part of its context).
@@ -319,60 +346,54 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int64_t s0 = token_slot(rowp, 0, a.page_size, a.num_slots, nullptr);
       dummy = s0 >= 0 ? static_cast<int32_t>(s0) : 0;
     }
-    // Slots of keys gw*64 + lane and gw*64 + 32 + lane of tile jj.
+    // Slots of keys u*32 + lane (u < 2) of step jj.
     auto lookup = [&](int jj, int32_t (&sl)[2]) {
 #pragma unroll
       for (int u = 0; u < 2; ++u) {
-        const int64_t key = static_cast<int64_t>(jj) * kKeysPerTile + gw * 64 + u * 32 + lane;
+        const int64_t key = static_cast<int64_t>(jj) * kKeysPerStep + u * 32 + lane;
         int64_t sv = -1;
-        if (jj < ntiles && key < kv_end && row_ok) sv = token_slot(rowp, key, a.page_size, a.num_slots, a.err);
+        if (jj < nsteps && key < kv_end && row_ok) sv = token_slot(rowp, key, a.page_size, a.num_slots, a.err);
         sl[u] = sv >= 0 ? static_cast<int32_t>(sv) : dummy;
       }
     };
-    auto copy_tile = [&](const uint8_t* base, uint32_t dst_tile, const int32_t (&sl)[2]) {
-#pragma unroll 8
-      for (int t = 0; t < 32; ++t) {
-        const int kl = 2 * t + h;  // key within this warp's 64
-        const int32_t slot = __shfl_sync(0xffffffffu, kl < 32 ? sl[0] : sl[1], kl & 31);
-        const int kk = gw * 64 + kl;  // key within the tile
-        const uint8_t* src = base + static_cast<int64_t>(slot) * a.slot_stride_bytes + g * 256 + c * 16;
-        const uint32_t dst = dst_tile + (c >> 3) * kHalfBytes + kk * 128 + (((c & 7) ^ (kk & 7)) << 4);
-        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+    auto copy_step = [&](const uint8_t* base, uint32_t dst_tile, const int32_t (&sl)[2]) {
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+#pragma unroll
+        for (int t = 0; t < 16; ++t) {
+          const int kk = u * 32 + 2 * t + h;  // key within the step
+          const int32_t slot = __shfl_sync(0xffffffffu, sl[u], 2 * t + h);
+          const uint8_t* src = base + static_cast<int64_t>(slot) * a.slot_stride_bytes + g * 256 + c * 16;
+          const uint32_t dst = dst_tile + (c >> 3) * kKvHalfBytes + kk * 128 + (((c & 7) ^ (kk & 7)) << 4);
+          asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+        }
       }
       asm volatile("cp.async.commit_group;" ::: "memory");
     };
-    const uint32_t k_dst = smem_u32(sK + grp * kTileBytes);
-    const uint32_t v_dst = smem_u32(sV + grp * kTileBytes);
     int32_t sl[2];
-    lookup(grp, sl);
-    for (int j = grp; j < ntiles; j += 2) {
-      const int use = j >> 1;
+    lookup(par, sl);
+    for (int j = par; j < nsteps; j += 2) {
+      const int st = j % kKvStages, use = j / kKvStages;
       if (use >= 1) {
-        const bool w = mbar_wait(&bars[kBarKEmpty + grp], (use - 1) & 1);
+        const bool w = mbar_wait(&bars[kBarKEmpty + st], (use - 1) & 1) &&
+                       mbar_wait(&bars[kBarVEmpty + st], (use - 1) & 1);
         if (__any_sync(0xffffffffu, !w || *abort_flag != 0)) {
           if (lane == 0 && !w) set_err(a.err, PKV_DEV_ERR_TIMEOUT);
           *abort_flag = 1;
           break;
         }
       }
-      copy_tile(a.kbase, k_dst, sl);
-      asm volatile("cp.async.wait_group 0;" ::: "memory");
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      mbar_arrive(&bars[kBarKFull + grp]);
-      if (use >= 1) {
-        const bool w = mbar_wait(&bars[kBarVEmpty + grp], (use - 1) & 1);
-        if (__any_sync(0xffffffffu, !w || *abort_flag != 0)) {
-          if (lane == 0 && !w) set_err(a.err, PKV_DEV_ERR_TIMEOUT);
-          *abort_flag = 1;
-          break;
-        }
-      }
-      copy_tile(a.vbase, v_dst, sl);
+      // K and V copies of the step fly together; K is signalled first.
+      copy_step(a.kbase, smem_u32(sK + st * kKvTileBytes), sl);
+      copy_step(a.vbase, smem_u32(sV + st * kKvTileBytes), sl);
       int32_t nsl[2];
-      lookup(j + 2, nsl);  // next tile's slots load while these copies fly
+      lookup(j + 2, nsl);  // this warp's next step; the loads fly with the copies
+      asm volatile("cp.async.wait_group 1;" ::: "memory");
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      mbar_arrive(&bars[kBarKFull + st]);
       asm volatile("cp.async.wait_group 0;" ::: "memory");
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      mbar_arrive(&bars[kBarVFull + grp]);
+      mbar_arrive(&bars[kBarVFull + st]);
       sl[0] = nsl[0];
       sl[1] = nsl[1];
     }
@@ -380,78 +401,100 @@ __global__ void __launch_bounds__(kThreads, 1)
     asm volatile("cp.async.wait_all;" ::: "memory");
   } else if (warp == kWarpMma) {
     // ============================ Q load + MMA issue ==========================
-    if (lane == 0) {
-      mbar_arrive_expect_tx(&bars[kBarQFull], kQTiles * kTileBytes);
+    // Step j writes S_i half (j % 2).  Issue order: QK_0(0), QK_1(0), QK_0(1),
+    // QK_1(1), then per step PV_0(j), QK_0(j+2), PV_1(j), QK_1(j+2): the scores
+    // for the next step are always computed before the softmax needs them, and
+    // QK_i(j+2) reuses the S half that PV_i(j) has just read P from (the
+    // tensor pipe executes in issue order).  The whole warp runs this loop so
+    // that descriptors and TMEM addresses stay warp-uniform (uniform
+    // registers); one elected lane issues each tcgen05 instruction.
+    if (elect_one()) {
+      mbar_arrive_expect_tx(&bars[kBarQFull], kQTiles * kQTileBytes);
       for (int i = 0; i < kQTiles; ++i)
-        for (int h = 0; h < 2; ++h)
-          tma_load_3d(sQ + i * kTileBytes + h * kHalfBytes, &qmap, h * 64, g * G,
+        for (int hh = 0; hh < 2; ++hh)
+          tma_load_3d(sQ + i * kQTileBytes + hh * kQHalfBytes, &qmap, hh * 64, g * G,
                       static_cast<int>(qbase + i0 + i * TQ), &bars[kBarQFull]);
-      const uint32_t q_addr = smem_u32(sQ);
-      const uint32_t k_addr = smem_u32(sK);
-      const uint32_t v_addr = smem_u32(sV);
-      bool ok = mbar_wait(&bars[kBarQFull], 0);
-      auto issue_qk = [&](int i, int st) {
-        const uint32_t d = tmem + kColS + 128 * i;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
-          const uint64_t ad = smem_desc(q_addr + i * kTileBytes + off, 16, 1024);
-          const uint64_t bd = smem_desc(k_addr + st * kTileBytes + off, 16, 1024);
-          mma_ss(d, ad, bd, kIdescQK, kk > 0 ? 1u : 0u);
-        }
-      };
-      auto issue_pv = [&](int i, int st, bool first) {
-        const uint32_t d = tmem + kColO + 128 * i;
-        const uint32_t pa = tmem + kColS + 128 * i;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t bd = smem_desc(v_addr + st * kTileBytes + kk * 2048, kHalfBytes, 1024);
-          mma_ts(d, pa + kk * 8, bd, kIdescPV, (first && kk == 0) ? 0u : 1u);
-        }
-      };
-      if (ok) ok = mbar_wait(&bars[kBarKFull + 0], 0);
-      if (ok) {
-        tc_fence_after();
-        issue_qk(0, 0);
-        mma_commit(&bars[kBarSFull + 0]);
-        issue_qk(1, 0);
-        mma_commit(&bars[kBarSFull + 1]);
-        mma_commit(&bars[kBarKEmpty + 0]);
-      }
-      for (int j = 0; j < ntiles && ok; ++j) {
-        const int st = j & 1, use = j >> 1;
-        const int st1 = (j + 1) & 1, use1 = (j + 1) >> 1;
-        ok = mbar_wait(&bars[kBarVFull + st], use & 1) && mbar_wait(&bars[kBarPReady + 0], j & 1);
-        if (!ok || *abort_flag) break;
-        tc_fence_after();
-        issue_pv(0, st, j == 0);
-        if (j + 1 < ntiles) {
-          ok = mbar_wait(&bars[kBarKFull + st1], use1 & 1);
-          if (!ok) break;
-          tc_fence_after();
-          issue_qk(0, st1);
-          mma_commit(&bars[kBarSFull + 0]);
-        }
-        ok = mbar_wait(&bars[kBarPReady + 1], j & 1);
-        if (!ok || *abort_flag) break;
-        tc_fence_after();
-        issue_pv(1, st, j == 0);
-        mma_commit(&bars[kBarVEmpty + st]);
-        if (j + 1 < ntiles) {
-          issue_qk(1, st1);
-          mma_commit(&bars[kBarSFull + 1]);
-          mma_commit(&bars[kBarKEmpty + st1]);
-        }
-      }
-      if (!ok) {
-        set_err(a.err, PKV_DEV_ERR_TIMEOUT);
-        *abort_flag = 1;
-      }
-      // Final commit: O complete (or, after an abort, every issued MMA retired).
-      mma_commit(&bars[kBarOFinal]);
-      if (!mbar_wait(&bars[kBarOFinal], 0)) set_err(a.err, PKV_DEV_ERR_TIMEOUT);
     }
     __syncwarp();
+    // Descriptor bases; k-steps add their byte offset / 16 to the start field.
+    const uint64_t q_desc = smem_desc(smem_u32(sQ), 16, 1024);
+    const uint64_t k_desc = smem_desc(smem_u32(sK), 16, 1024);
+    const uint64_t v_desc = smem_desc(smem_u32(sV), kKvHalfBytes, 1024);
+    auto issue_qk = [&](int i, int j) {
+      const uint32_t d = tmem + kColS + 128 * i + 64 * (j & 1);
+      const uint64_t ad = q_desc + static_cast<uint64_t>((i * kQTileBytes) >> 4);
+      const uint64_t bd = k_desc + static_cast<uint64_t>(((j % kKvStages) * kKvTileBytes) >> 4);
+      if (elect_one()) {
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint64_t ao = static_cast<uint64_t>(((kk >> 2) * kQHalfBytes + (kk & 3) * 32) >> 4);
+          const uint64_t bo = static_cast<uint64_t>(((kk >> 2) * kKvHalfBytes + (kk & 3) * 32) >> 4);
+          mma_ss(d, ad + ao, bd + bo, kIdescQK, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(&bars[kBarSFull + 2 * i + (j & 1)]);
+      }
+      __syncwarp();
+    };
+    auto issue_pv = [&](int i, int j) {
+      const uint32_t d = tmem + kColO + 128 * i;
+      const uint32_t pa = tmem + kColS + 128 * i + 64 * (j & 1);
+      const uint64_t bd = v_desc + static_cast<uint64_t>(((j % kKvStages) * kKvTileBytes) >> 4);
+      if (elect_one()) {
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_ts(d, pa + kk * 8, bd + static_cast<uint64_t>((kk * 2048) >> 4), kIdescPV,
+                 (j == 0 && kk == 0) ? 0u : 1u);
+        mma_commit(&bars[kBarODone + i]);
+      }
+      __syncwarp();
+    };
+    auto commit = [&](int bar) {
+      if (elect_one()) mma_commit(&bars[bar]);
+      __syncwarp();
+    };
+    auto wait_all = [&](int bar, uint32_t parity) -> bool {
+      return __all_sync(0xffffffffu, mbar_wait(&bars[bar], parity));
+    };
+    bool ok = wait_all(kBarQFull, 0);
+    for (int j = 0; j < 2 && j < nsteps && ok; ++j) {
+      ok = wait_all(kBarKFull + j, 0);
+      if (!ok) break;
+      tc_fence_after();
+      issue_qk(0, j);
+      issue_qk(1, j);
+      commit(kBarKEmpty + j);
+    }
+    for (int j = 0; j < nsteps && ok; ++j) {
+      const int st = j % kKvStages, use = j / kKvStages;
+      const bool more = j + 2 < nsteps;
+      const int st2 = (j + 2) % kKvStages, use2 = (j + 2) / kKvStages;
+      ok = wait_all(kBarVFull + st, use & 1) && wait_all(kBarPReady + 0 + (j & 1), (j >> 1) & 1);
+      if (!ok || __any_sync(0xffffffffu, *abort_flag != 0)) break;
+      tc_fence_after();
+      issue_pv(0, j);
+      if (more) {
+        ok = wait_all(kBarKFull + st2, use2 & 1);
+        if (!ok) break;
+        tc_fence_after();
+        issue_qk(0, j + 2);
+      }
+      ok = wait_all(kBarPReady + 2 + (j & 1), (j >> 1) & 1);
+      if (!ok || __any_sync(0xffffffffu, *abort_flag != 0)) break;
+      tc_fence_after();
+      issue_pv(1, j);
+      commit(kBarVEmpty + st);
+      if (more) {
+        issue_qk(1, j + 2);
+        commit(kBarKEmpty + st2);
+      }
+    }
+    if (!ok) {
+      if (lane == 0) set_err(a.err, PKV_DEV_ERR_TIMEOUT);
+      *abort_flag = 1;
+    }
+    // Final commit: O complete (or, after an abort, every issued MMA retired).
+    commit(kBarOFinal);
+    if (!wait_all(kBarOFinal, 0) && lane == 0) set_err(a.err, PKV_DEV_ERR_TIMEOUT);
   } else if (warp < kWarpLoad0) {
     // ============================ softmax + epilogue ==========================
     const int i = warp >> 2;         // Q tile
@@ -462,38 +505,40 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool valid = tok < e;
     const int64_t lim = valid ? static_cast<int64_t>(p) + tok + 1 : 1;  // keys < lim visible
     const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
-    const uint32_t s_addr = tmem + lane_base + kColS + 128 * i;
     const uint32_t o_addr = tmem + lane_base + kColO + 128 * i;
     float m_run = -INFINITY;
     float2 l2 = make_float2(0.f, 0.f);  // running sum of p, even / odd keys
     const float2 sl2 = make_float2(a.scale_log2, a.scale_log2);
     bool ok = true;
-    for (int j = 0; j < ntiles; ++j) {
-      const bool w = mbar_wait(&bars[kBarSFull + i], j & 1);
+    for (int j = 0; j < nsteps; ++j) {
+      const int hf = j & 1;
+      const uint32_t s_addr = tmem + lane_base + kColS + 128 * i + 64 * hf;
+      const bool w = mbar_wait(&bars[kBarSFull + 2 * i + hf], (j >> 1) & 1);
       if (__any_sync(0xffffffffu, !w || *abort_flag != 0)) { ok = false; break; }
       tc_fence_after();
-      const int64_t kb = static_cast<int64_t>(j) * kKeysPerTile;
-      // Keys kb .. kb + vis - 1 of this tile are visible to this row.
+      const int64_t kb = static_cast<int64_t>(j) * kKeysPerStep;
+      // Keys kb .. kb + vis - 1 of this step are visible to this row.
       const int64_t vis64 = lim - kb;
-      const int32_t vis = vis64 <= 0 ? 0 : (vis64 >= kKeysPerTile ? kKeysPerTile : static_cast<int32_t>(vis64));
-      const bool warp_full = __all_sync(0xffffffffu, vis == kKeysPerTile);
-      // ---- pass 1: row max of the raw scores ----
+      const int32_t vis = vis64 <= 0 ? 0 : (vis64 >= kKeysPerStep ? kKeysPerStep : static_cast<int32_t>(vis64));
+      const bool warp_full = __all_sync(0xffffffffu, vis == kKeysPerStep);
+      uint32_t sr[64];
+      tmem_ld64_nowait(s_addr, sr);
+      tmem_wait_ld();
       float mx = -INFINITY;
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        float v[32];
-        tmem_ld32(s_addr + c * 32, v);
-        if (warp_full) {
+      if (warp_full) {
 #pragma unroll
-          for (int u = 0; u < 32; u += 2) mx = max3f(mx, v[u], v[u + 1]);
-        } else {
+        for (int u = 0; u < 64; u += 2) mx = max3f(mx, __uint_as_float(sr[u]), __uint_as_float(sr[u + 1]));
+      } else {
 #pragma unroll
-          for (int u = 0; u < 32; ++u) mx = (c * 32 + u < vis) ? fmaxf(mx, v[u]) : mx;
-        }
+        for (int u = 0; u < 64; ++u) mx = (u < vis) ? fmaxf(mx, __uint_as_float(sr[u])) : mx;
       }
       mx *= a.scale_log2;
       const bool need = mx > m_run + kRescaleThreshold;
       if (j > 0 && __any_sync(0xffffffffu, need)) {
+        // O holds PV of steps < j; wait until the last of them has retired.
+        const bool wo = mbar_wait(&bars[kBarODone + i], (j - 1) & 1);
+        if (__any_sync(0xffffffffu, !wo)) { ok = false; break; }
+        tc_fence_after();
         const float alpha = need ? ex2_approx(m_run - mx) : 1.f;
         l2.x *= alpha;
         l2.y *= alpha;
@@ -509,16 +554,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (need) m_run = mx;
       const float2 negm2 = make_float2(-m_run, -m_run);
-      // ---- pass 2: p = 2^(s * scale * log2e - m), packed to bf16 over S ----
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        float v[32];
-        tmem_ld32(s_addr + c * 32, v);
+      // p = 2^(s * scale * log2e - m), packed to bf16 over the half's first 32 columns.
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
         uint32_t w16[16];
         if (warp_full) {
 #pragma unroll
           for (int u = 0; u < 32; u += 2) {
-            const float2 t = __ffma2_rn(make_float2(v[u], v[u + 1]), sl2, negm2);
+            const float2 t = __ffma2_rn(make_float2(__uint_as_float(sr[32 * c + u]), __uint_as_float(sr[32 * c + u + 1])),
+                                        sl2, negm2);
             const float2 pp = make_float2(ex2_approx(t.x), ex2_approx(t.y));
             l2 = __fadd2_rn(l2, pp);
             w16[u >> 1] = pack_bf16x2(pp.x, pp.y);
@@ -526,18 +570,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else {
 #pragma unroll
           for (int u = 0; u < 32; u += 2) {
-            const float2 t = __ffma2_rn(make_float2(v[u], v[u + 1]), sl2, negm2);
-            const float p0 = (c * 32 + u < vis) ? ex2_approx(t.x) : 0.f;
-            const float p1 = (c * 32 + u + 1 < vis) ? ex2_approx(t.y) : 0.f;
+            const float2 t = __ffma2_rn(make_float2(__uint_as_float(sr[32 * c + u]), __uint_as_float(sr[32 * c + u + 1])),
+                                        sl2, negm2);
+            const float p0 = (32 * c + u < vis) ? ex2_approx(t.x) : 0.f;
+            const float p1 = (32 * c + u + 1 < vis) ? ex2_approx(t.y) : 0.f;
             l2 = __fadd2_rn(l2, make_float2(p0, p1));
             w16[u >> 1] = pack_bf16x2(p0, p1);
           }
         }
-        tmem_st16(s_addr + c * 16, w16);
+        tmem_st16(s_addr + 16 * c, w16);
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&bars[kBarPReady + i]);
+      mbar_arrive(&bars[kBarPReady + 2 * i + hf]);
     }
     const float l_run = l2.x + l2.y;
     if (!ok && lane == 0) {
