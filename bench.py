@@ -61,15 +61,16 @@ def source_hash(*names):
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(kernel: str, src_hash: str):
+def recorded_traffic(kernel: str, src_hash: str, workload: str):
     """Per-launch DRAM bytes of `kernel` from the committed ncu summary, or None
-    when the kernel's source has changed since the counters were taken."""
+    when the kernel's source has changed since the counters were taken or the
+    capture was of another workload."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(p) as f:
             d = json.load(f)
         e = d.get(kernel)
-        if e and e.get("source_hash") == src_hash:
+        if e and e.get("source_hash") == src_hash and e.get("workload") == workload:
             return float(e["dram_bytes_per_launch"])
     except Exception:
         pass
@@ -314,7 +315,7 @@ def run_decode(args, world, rank, local):
     hbm, bf16, bf16s, peak_src = measured_peaks()
     dec_avg_ms = sum(dec_ms) / len(dec_ms)
     achieved = per_call / (dec_avg_ms / 1e3) / 1e9
-    traffic = recorded_traffic("decode_split_kernel", source_hash("decode.cu", "common.cuh"))
+    traffic = recorded_traffic("decode_split_kernel", source_hash("decode.cu", "common.cuh"), wl.name)
 
     # ---- e2e through the C ABI with host buffers -------------------------------
     import torch as _t
@@ -381,7 +382,7 @@ def run_decode(args, world, rank, local):
             "l2": "inputs larger than L2 (no flush)",
             "parallelism": f"replicas x{world}",
         },
-        "decode_tok_per_s_per_layer": round(world * wl.batch * args.steps * nL / (ms_total / 1e3) / nL, 1),
+        "decode_tok_per_s_per_layer": round(world * wl.batch * args.steps * nL / (ms_total / 1e3), 1),
         "decode_call_us": round(dec_avg_ms * 1e3, 2),
         "store_kv_call_us": round(sum(st_ms) / len(st_ms) * 1e3, 2),
         "roofline": {
@@ -457,8 +458,230 @@ def run_extend_measure(dev, warmup=3, iters=10):
     return {"workload": "chunked-prefill extend, 2048-token chunk at prefix 6144, Hq 32 Hkv 8",
             "tflops": round(tf, 2), "ms": round(med, 4), "flops": flops,
             "roofline": {"bound": "tensor", "achieved": round(tf, 2), "peak": bf16,
-                         "peak_source": src, "unit": "TFLOP/s", "frac": round(tf / bf16, 4)},
+                         "peak_source": src, "unit": "TFLOP/s", "frac": round(tf / bf16, 4),
+                         "traffic": recorded_traffic("extend_tc_kernel",
+                                                     source_hash("extend_tc.cu", "common.cuh"),
+                                                     "chunked-prefill extend c3")},
             "device_error_word": int(err.item())}
+
+
+def _dev_pool(W, api, torch, wl, dev, layers):
+    """Device pool for a workload: host plane contents copied to `layers`."""
+    spec = wl.pool
+    pool = api.KVPool.empty(spec.num_layers, spec.num_slots, spec.num_kv_heads,
+                            page_size=spec.page_size, device=dev)
+    src_layer = next(iter(wl.k_planes.keys()))
+    hk = torch.from_numpy(np.ascontiguousarray(wl.k_planes[src_layer]).view(np.int16)).view(torch.bfloat16).to(dev)
+    hv = torch.from_numpy(np.ascontiguousarray(wl.v_planes[src_layer]).view(np.int16)).view(torch.bfloat16).to(dev)
+    for l in layers:
+        pool.k[l].copy_(hk)
+        pool.v[l].copy_(hv)
+    return pool
+
+
+def _flops_extend(wl):
+    return 4 * 128 * wl.num_q_heads * wl.causal_pairs()
+
+
+def run_chunked_prefill(args, world, rank, local):
+    """One step = the four 2048-token chunks of one 8192-token prompt (prefix
+    0, 2048, 4096, 6144), each with its store_kv and the 128-request decode
+    batch at context 2048 (two calls per chunk on one stream)."""
+    import torch
+    from paged_kv_gqa_scatter_b200 import api
+    from paged_kv_gqa_scatter_b200 import workloads as W
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    mix = W.chunked_prefill_step(step=3)
+    ext, dec = mix.extend, mix.decode
+
+    def tdev(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    pool = _dev_pool(W, api, torch, ext, dev, [0])
+    table = api.PageTable(torch.from_numpy(ext.page_table).to(dev))
+    e_q, e_k, e_v = tdev(ext.q), tdev(ext.k_new), tdev(ext.v_new)
+    e_ti = torch.from_numpy(ext.table_idx).to(dev)
+    e_el = torch.from_numpy(ext.extend_lens).to(dev)
+    e_qo = torch.from_numpy(ext.q_offsets).to(dev)
+    row = ext.page_table[ext.table_idx[0]]
+    chunk = int(ext.extend_lens[0])
+    e_loc = [torch.from_numpy(row[c * chunk:(c + 1) * chunk].astype(np.int32)).to(dev) for c in range(4)]
+    e_pl = [torch.tensor([c * chunk], dtype=torch.int32, device=dev) for c in range(4)]
+    e_out = torch.empty_like(e_q)
+    d_q, d_k, d_v = tdev(dec.q), tdev(dec.k_new), tdev(dec.v_new)
+    d_ti = torch.from_numpy(dec.table_idx).to(dev)
+    d_sl = torch.from_numpy(dec.seq_lens).to(dev)
+    d_loc = torch.from_numpy(dec.out_loc).to(dev)
+    d_out = torch.empty_like(d_q)
+    ws = api.decode_workspace(dec.batch, dec.num_q_heads, device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    s = torch.cuda.current_stream(dev)
+    evs = []
+
+    def step(record):
+        for c in range(4):
+            es = [torch.cuda.Event(enable_timing=True) for _ in range(3)] if record else None
+            api.store_kv(pool, 0, e_k, e_v, e_loc[c], err)
+            api.store_kv(pool, 0, d_k, d_v, d_loc, err)
+            if record: es[0].record(s)
+            api.extend_attn(pool, 0, e_q, table, e_ti, e_pl[c], e_el, e_qo, chunk, e_out,
+                            scale=ext.scale, dev_err=err)
+            if record: es[1].record(s)
+            api.decode_attn(pool, 0, d_q, table, d_ti, d_sl, d_out, ws, scale=dec.scale, dev_err=err)
+            if record:
+                es[2].record(s)
+                evs.append(es)
+
+    for _ in range(args.warmup):
+        step(False)
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks.start()
+    start.record(s)
+    for _ in range(args.steps):
+        step(True)
+    stop.record(s)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    ms = max_over_ranks(start.elapsed_time(stop), world)
+    ext_ms = sum(e[0].elapsed_time(e[1]) for e in evs)
+    dec_ms = sum(e[1].elapsed_time(e[2]) for e in evs)
+    pairs = sum(chunk * (c * chunk) + chunk * (chunk + 1) // 2 for c in range(4))
+    ext_flops = 4 * 128 * ext.num_q_heads * pairs * args.steps
+    dec_bytes = decode_bytes(dec) * 4 * args.steps
+    _, bf16, _, src = measured_peaks()
+    hbm, _, _, hsrc = measured_peaks()
+    tf = ext_flops / (ext_ms / 1e3) / 1e12
+    gbs = dec_bytes / (dec_ms / 1e3) / 1e9
+    return {
+        "metric": "chunked-prefill step: extend-attn TFLOP/s",
+        "value": round(world * tf, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded PCG64 N(0,1) values rounded to bf16)",
+        "config": {"workload": "chunked-prefill", "prompt": 8192, "chunk": chunk,
+                   "decode_batch": dec.batch, "decode_context": int(dec.seq_lens[0]),
+                   "num_q_heads": ext.num_q_heads, "num_kv_heads": ext.pool.num_kv_heads,
+                   "step": "4 chunks x (store_kv chunk + decode rows, extend_attn, decode_attn)",
+                   "parallelism": f"replicas x{world}"},
+        "extend": {"tflops": round(tf, 2), "ms_per_step": round(ext_ms / args.steps, 4),
+                   "roofline": {"bound": "tensor", "achieved": round(tf, 2), "peak": bf16,
+                                "peak_source": src, "unit": "TFLOP/s", "frac": round(tf / bf16, 4)}},
+        "decode": {"gbs": round(gbs, 1), "ms_per_step": round(dec_ms / args.steps, 4),
+                   "tok_per_s_per_layer": round(dec.batch * 4 * args.steps / (dec_ms / 1e3), 1),
+                   "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm,
+                                "peak_source": hsrc, "unit": "GB/s", "frac": round(gbs / hbm, 4)}},
+        "gpu_launches": args.steps * 4 * 5,
+        "device_error_word": int(err.item()),
+        "clocks": clk,
+    }
+
+
+def run_radix(args, world, rank, local):
+    """Radix shared-prefix serving on a 32-layer pool: one step = the extend of
+    all 256 suffixes on every layer (store_kv + extend_attn per layer), then
+    decode step 1 on every layer (store_kv + decode_attn per layer)."""
+    import torch
+    from paged_kv_gqa_scatter_b200 import api
+    from paged_kv_gqa_scatter_b200 import workloads as W
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    rs = W.radix_shared_prefix()
+    ext = rs.extend
+    dec = rs.decode_step(1)
+    L = ext.pool.num_layers
+
+    def tdev(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    pool = _dev_pool(W, api, torch, ext, dev, range(L))
+    table = api.PageTable(torch.from_numpy(ext.page_table).to(dev))
+    e_q, e_k, e_v = tdev(ext.q), tdev(ext.k_new), tdev(ext.v_new)
+    e_ti = torch.from_numpy(ext.table_idx).to(dev)
+    e_pl = torch.from_numpy(ext.prefix_lens).to(dev)
+    e_el = torch.from_numpy(ext.extend_lens).to(dev)
+    e_qo = torch.from_numpy(ext.q_offsets).to(dev)
+    e_loc = torch.from_numpy(ext.out_loc).to(dev)
+    e_out = torch.empty_like(e_q)
+    mx = int(ext.extend_lens.max())
+    d_q, d_k, d_v = tdev(dec.q), tdev(dec.k_new), tdev(dec.v_new)
+    d_ti = torch.from_numpy(dec.table_idx).to(dev)
+    d_sl = torch.from_numpy(dec.seq_lens).to(dev)
+    d_loc = torch.from_numpy(dec.out_loc).to(dev)
+    d_out = torch.empty_like(d_q)
+    ws = api.decode_workspace(dec.batch, dec.num_q_heads, device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    s = torch.cuda.current_stream(dev)
+    ext_ev, dec_ev = [], []
+
+    def step(record):
+        for l in range(L):
+            api.store_kv(pool, l, e_k, e_v, e_loc, err)
+            a = torch.cuda.Event(enable_timing=True) if record else None
+            b = torch.cuda.Event(enable_timing=True) if record else None
+            if record: a.record(s)
+            api.extend_attn(pool, l, e_q, table, e_ti, e_pl, e_el, e_qo, mx, e_out, scale=ext.scale, dev_err=err)
+            if record:
+                b.record(s)
+                ext_ev.append((a, b))
+        for l in range(L):
+            api.store_kv(pool, l, d_k, d_v, d_loc, err)
+            a = torch.cuda.Event(enable_timing=True) if record else None
+            b = torch.cuda.Event(enable_timing=True) if record else None
+            if record: a.record(s)
+            api.decode_attn(pool, l, d_q, table, d_ti, d_sl, d_out, ws, scale=dec.scale, dev_err=err)
+            if record:
+                b.record(s)
+                dec_ev.append((a, b))
+
+    for _ in range(args.warmup):
+        step(False)
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks.start()
+    start.record(s)
+    for _ in range(args.steps):
+        step(True)
+    stop.record(s)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    ms = max_over_ranks(start.elapsed_time(stop), world)
+    ext_ms = sum(a.elapsed_time(b) for a, b in ext_ev)
+    dec_ms = sum(a.elapsed_time(b) for a, b in dec_ev)
+    ext_flops = _flops_extend(ext) * L * args.steps
+    logical = decode_bytes(dec) * L * args.steps
+    _, bf16, _, src = measured_peaks()
+    hbm, _, _, hsrc = measured_peaks()
+    tf = ext_flops / (ext_ms / 1e3) / 1e12
+    return {
+        "metric": "radix shared-prefix: extend-attn TFLOP/s",
+        "value": round(world * tf, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded PCG64 N(0,1) values rounded to bf16; per-layer inputs reused)",
+        "config": {"workload": "radix-prefix", "layers": L, "batch": ext.batch, "prefix": 4096,
+                   "suffix_tokens": ext.total_q, "num_q_heads": ext.num_q_heads,
+                   "num_kv_heads": ext.pool.num_kv_heads,
+                   "step": "per layer store_kv + extend_attn, then per layer store_kv + decode_attn (decode step 1)",
+                   "parallelism": f"replicas x{world}"},
+        "extend": {"tflops": round(tf, 2), "ms_per_layer": round(ext_ms / (L * args.steps), 4),
+                   "roofline": {"bound": "tensor", "achieved": round(tf, 2), "peak": bf16,
+                                "peak_source": src, "unit": "TFLOP/s", "frac": round(tf / bf16, 4)}},
+        "decode": {"ms_per_layer": round(dec_ms / (L * args.steps), 4),
+                   "tok_per_s_per_layer": round(dec.batch * L * args.steps / (dec_ms / 1e3), 1),
+                   "logical_gbs": round(logical / (dec_ms / 1e3) / 1e9, 1),
+                   "note": "logical bytes count the shared 4096-token prefix once per request; most of it is served from L2"},
+        "gpu_launches": args.steps * L * 5,
+        "device_error_word": int(err.item()),
+        "clocks": clk,
+    }
 
 
 # ---------------------------------------------------------------------------
@@ -510,7 +733,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="decode-qwen3-0.6b",
-                    choices=["decode-qwen3-0.6b", "decode-qwen3-8b"])
+                    choices=["decode-qwen3-0.6b", "decode-qwen3-8b", "chunked-prefill", "radix-prefix"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--pool-layers", type=int, default=28,
                     help="layers of the decode-qwen3-0.6b pool (28 as stated; fewer only for profiling)")
@@ -526,7 +749,12 @@ def main():
             print(json.dumps(res), flush=True)
         return 0
     world, rank, local = dist_setup()
-    res = run_decode(args, world, rank, local)
+    if args.workload == "chunked-prefill":
+        res = run_chunked_prefill(args, world, rank, local)
+    elif args.workload == "radix-prefix":
+        res = run_radix(args, world, rank, local)
+    else:
+        res = run_decode(args, world, rank, local)
     if rank == 0:
         print(json.dumps(res), flush=True)
     if world > 1:
