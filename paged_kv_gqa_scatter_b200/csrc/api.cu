@@ -57,6 +57,7 @@ int check_pool(const pkv_pool* p, int32_t layer, PoolView* out) {
 int check_table(const pkv_page_table* t, TableView* out) {
   if (t == nullptr || t->entries == nullptr) return PKV_ERR_INVALID_ARG;
   if (t->rows < 1 || t->cols < 1 || t->row_stride < t->cols) return PKV_ERR_INVALID_ARG;
+  if (t->cols > INT_MAX) return PKV_ERR_TOO_LARGE;
   out->entries = t->entries;
   out->rows = t->rows;
   out->cols = t->cols;

@@ -154,23 +154,33 @@ __device__ __forceinline__ uint64_t policy_evict_last() {
 }
 
 // ---- page table -----------------------------------------------------------
+// Offset of token (or slot) j inside its page of P tokens: a mask when P is a
+// power of two, else a 32-bit remainder.  Token positions and table entries are
+// 32-bit (the host rejects tables wider than 2^31 columns).
+__device__ __forceinline__ int32_t page_offset(int32_t j, int32_t page_size) {
+  return (page_size & (page_size - 1)) == 0 ? (j & (page_size - 1)) : (j % page_size);
+}
+
 // Slot of token j of the request in table row `row` (row already checked).
-// page_size 1: the entry.  page_size P > 1: entry at column P*(j/P), divided
-// by P, is the page; the slot is page*P + j%P.  Returns -1 (and sets an error
-// bit) when the entry is out of range or not page aligned.
-__device__ __forceinline__ int64_t token_slot(const int32_t* __restrict__ row_ptr, int64_t j,
+// page_size 1: the entry.  page_size P > 1: the entry at column P*(j/P) is the
+// page's first slot (page id * P, so page = entry / P) and the slot is
+// page*P + j%P, i.e. entry + j%P.  Returns -1 (and sets an error bit) when the
+// entry is not page aligned or the slot is out of range.
+__device__ __forceinline__ int64_t token_slot(const int32_t* __restrict__ row_ptr, int64_t j64,
                                               int32_t page_size, int64_t num_slots,
                                               int32_t* err) {
+  const int32_t j = static_cast<int32_t>(j64);
   int64_t slot;
   if (page_size == 1) {
     slot = row_ptr[j];
   } else {
-    const int32_t e = row_ptr[(j / page_size) * page_size];
-    if (e % page_size != 0) {
+    const int32_t off = page_offset(j, page_size);
+    const int32_t e = row_ptr[j - off];
+    if (page_offset(e, page_size) != 0) {
       set_err(err, PKV_DEV_ERR_PAGE_ALIGN);
       return -1;
     }
-    slot = static_cast<int64_t>(e / page_size) * page_size + (j % page_size);
+    slot = static_cast<int64_t>(e) + off;
   }
   if (slot < 0 || slot >= num_slots) {
     set_err(err, PKV_DEV_ERR_SLOT_RANGE);

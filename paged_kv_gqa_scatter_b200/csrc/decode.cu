@@ -79,17 +79,13 @@ struct DecodeArgs {
 
 // Shared memory layout (bytes), identical on host and device.
 struct DecodeSmem {
-  int32_t scan_off, cum_off, psm_off, ring_off, stage_bytes, total;
+  int32_t cum_off, psm_off, ring_off, stage_bytes, total;
 };
-
-constexpr int kMaxThreads = 32 * 9;
 
 __host__ __device__ inline DecodeSmem decode_smem_layout(int batch, int hkv, int row_bytes, int T,
                                                          int G) {
   DecodeSmem L;
   int off = 2 * kStages * 8 + 16;  // full/empty barriers + abort flag
-  L.scan_off = off;
-  off += 4 * kMaxThreads;
   L.cum_off = off;
   off += 4 * (batch + 1);
   off = (off + 15) & ~15;
@@ -162,12 +158,13 @@ __global__ void __launch_bounds__(32 * 9, 1) decode_split_kernel(const DecodeArg
   }
 
   // ---- plan: prefix sums of clamped context lengths -------------------------
+  // One warp: each lane sums a contiguous segment of requests, one shuffle
+  // scan combines the segments, and each lane writes its segment's prefixes.
   const int B = a.batch;
   const int nthr = blockDim.x;
-  {
-    int32_t* scan = reinterpret_cast<int32_t*>(smem + L.scan_off);
-    const int seg = (B + nthr - 1) / nthr;
-    const int r0 = min(B, static_cast<int>(threadIdx.x) * seg);
+  if (warp == 0) {
+    const int seg = (B + 31) >> 5;
+    const int r0 = min(B, lane * seg);
     const int r1 = min(B, r0 + seg);
     int32_t ssum = 0;
     for (int r = r0; r < r1; ++r) {
@@ -180,31 +177,20 @@ __global__ void __launch_bounds__(32 * 9, 1) decode_split_kernel(const DecodeArg
       cum[r + 1] = n;
       ssum += n;
     }
-    scan[threadIdx.x] = ssum;
-    __syncthreads();
-    if (warp == 0) {
-      int32_t carry = 0;
-      for (int base = 0; base < nthr; base += 32) {
-        const int32_t x0 = (base + lane < nthr) ? scan[base + lane] : 0;
-        int32_t x = x0;
+    int32_t x = ssum;
 #pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-          const int32_t y = __shfl_up_sync(0xffffffffu, x, off);
-          if (lane >= off) x += y;
-        }
-        if (base + lane < nthr) scan[base + lane] = carry + x - x0;
-        carry += __shfl_sync(0xffffffffu, x, 31);
-      }
+    for (int off = 1; off < 32; off <<= 1) {
+      const int32_t y = __shfl_up_sync(0xffffffffu, x, off);
+      if (lane >= off) x += y;
     }
-    __syncthreads();
-    int32_t run = scan[threadIdx.x];
+    int32_t run = x - ssum;  // exclusive prefix of this lane's segment
     for (int r = r0; r < r1; ++r) {
       run += cum[r + 1];
       cum[r + 1] = run;
     }
-    if (threadIdx.x == 0) cum[0] = 0;
-    __syncthreads();
+    if (lane == 0) cum[0] = 0;
   }
+  __syncthreads();
   const int64_t total = cum[B];
   int64_t per = (total + gridDim.x - 1) / gridDim.x;
   if (per < kMinTokensPerCta) per = kMinTokensPerCta;
@@ -266,7 +252,8 @@ __global__ void __launch_bounds__(32 * 9, 1) decode_split_kernel(const DecodeArg
     auto lookup = [&](const Cursor& c, bool have) -> int32_t {
       const int64_t j = c.j0 + lane;
       if (!have || lane >= T || j >= c.jb || !c.row_ok) return 0;
-      return a.page_size == 1 ? c.rowp[j] : c.rowp[(j / a.page_size) * a.page_size];
+      const int32_t j32 = static_cast<int32_t>(j);
+      return a.page_size == 1 ? c.rowp[j32] : c.rowp[j32 - page_offset(j32, a.page_size)];
     };
     Cursor c0{}, c1{}, c2{};
     bool h0 = piece_start(rfirst, c0);
@@ -304,8 +291,8 @@ __global__ void __launch_bounds__(32 * 9, 1) decode_split_kernel(const DecodeArg
         bool aligned = true;
         if (a.page_size == 1) {
           slot = e0;
-        } else if (e0 % a.page_size == 0) {
-          slot = static_cast<int64_t>(e0 / a.page_size) * a.page_size + (j % a.page_size);
+        } else if (page_offset(e0, a.page_size) == 0) {
+          slot = static_cast<int64_t>(e0) + page_offset(static_cast<int32_t>(j), a.page_size);
         } else {
           aligned = false;
           set_err(a.err, PKV_DEV_ERR_PAGE_ALIGN);
@@ -367,6 +354,10 @@ __global__ void __launch_bounds__(32 * 9, 1) decode_split_kernel(const DecodeArg
     const int64_t jb = min(hi, (int64_t)cum[r + 1]) - cum[r];
     if (jb <= ja) continue;
     const bool whole = cum[r] >= lo && cum[r + 1] <= hi;
+    // Warm L2 with the next request's queries while this piece runs.
+    if (r + 1 < B && cum[r + 1] < hi && lane < 2 * G)
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(qbase + ((int64_t)(r + 1) * a.hq + g * G) * kHeadDim +
+                                                      lane * (128 / ESZ)));
 
     float2 q2[G][4];
 #pragma unroll
@@ -552,22 +543,22 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(
   const int64_t per = *per_p;
   const int64_t k_lo = c0 / per, k_hi = (c1 - 1) / per;
   if (k_lo == k_hi) return;  // written by its only piece
-  float M = -INFINITY;
-  for (int64_t k = k_lo + lane; k <= k_hi; k += 32) M = fmaxf(M, ml[(k + r) * hq + h].x);
-#pragma unroll
-  for (int off = 16; off >= 1; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+  // Online merge: the loads of consecutive pieces are independent, so the
+  // unrolled loop keeps several in flight.
+  float M = -INFINITY, den = 0.f;
   float4 acc = make_float4(0, 0, 0, 0);
-  float den = 0.f;
 #pragma unroll 4
   for (int64_t k = k_lo; k <= k_hi; ++k) {
     const float2 st = ml[(k + r) * hq + h];
     const float4 x = *reinterpret_cast<const float4*>(o + ((k + r) * hq + h) * kHeadDim + 4 * lane);
-    const float w = exp2f(st.x - M);
-    den += w * st.y;
-    acc.x += w * x.x;
-    acc.y += w * x.y;
-    acc.z += w * x.z;
-    acc.w += w * x.w;
+    const float Mn = fmaxf(M, st.x);
+    const float wa = exp2f(M - Mn), wb = exp2f(st.x - Mn);
+    den = den * wa + wb * st.y;
+    acc.x = acc.x * wa + wb * x.x;
+    acc.y = acc.y * wa + wb * x.y;
+    acc.z = acc.z * wa + wb * x.z;
+    acc.w = acc.w * wa + wb * x.w;
+    M = Mn;
   }
   const float inv = den > 0.f ? 1.f / den : 0.f;
   if constexpr (sizeof(E) == 2) {
