@@ -154,13 +154,20 @@ def barrier(world):
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """Largest value of x over the ranks (device time is taken as the slowest rank)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(units_per_rank_step: float, steps: int, ms_max: float, world: int) -> float:
+    """Whole-job rate: the units every rank processed over the slowest rank's time (units/s)."""
+    return world * units_per_rank_step * steps / (ms_max / 1e3)
 
 
 def blas_threads():
@@ -311,7 +318,7 @@ def run_decode(args, world, rank, local):
 
     per_call = decode_bytes(wl)
     step_bytes = nL * (per_call + store_bytes(wl))
-    value = world * step_bytes * args.steps / (ms_total / 1e3) / 1e9
+    value = job_throughput(step_bytes, args.steps, ms_total, world) / 1e9
     hbm, bf16, bf16s, peak_src = measured_peaks()
     dec_avg_ms = sum(dec_ms) / len(dec_ms)
     achieved = per_call / (dec_avg_ms / 1e3) / 1e9
@@ -355,7 +362,7 @@ def run_decode(args, world, rank, local):
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
-    e2e_val = world * step_bytes * args.steps / (e2e_ms / 1e3) / 1e9
+    e2e_val = job_throughput(step_bytes, args.steps, e2e_ms, world) / 1e9
 
     result = {
         "metric": "paged decode-attn KV GB/s",
