@@ -364,6 +364,28 @@ def run_decode(args, world, rank, local):
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
     e2e_val = job_throughput(step_bytes, args.steps, e2e_ms, world) / 1e9
 
+    # ---- the same step replayed from a CUDA graph (fixed buffers) ---------------
+    graph_us = None
+    try:
+        gs = torch.cuda.Stream(dev)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=gs):
+            step()
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize()
+        g0 = torch.cuda.Event(enable_timing=True)
+        g1 = torch.cuda.Event(enable_timing=True)
+        g0.record(stream)
+        for _ in range(args.steps):
+            g.replay()
+        g1.record(stream)
+        torch.cuda.synchronize()
+        graph_us = round(g0.elapsed_time(g1) / args.steps * 1e3, 2)
+        del g
+    except Exception as exc:  # reported, not hidden: the field says why it is missing
+        graph_us = f"unavailable: {type(exc).__name__}: {exc}"[:200]
+
     result = {
         "metric": "paged decode-attn KV GB/s",
         "value": round(value, 2),
@@ -392,6 +414,7 @@ def run_decode(args, world, rank, local):
         "decode_tok_per_s_per_layer": round(world * wl.batch * args.steps * nL / (ms_total / 1e3), 1),
         "decode_call_us": round(dec_avg_ms * 1e3, 2),
         "store_kv_call_us": round(sum(st_ms) / len(st_ms) * 1e3, 2),
+        "graph_step_us": graph_us,
         "roofline": {
             "kernel": "decode_attn (decode_split_kernel + decode_combine_kernel, timed together)",
             "bound": "hbm",

@@ -575,8 +575,11 @@ template <typename E, int G>
 cudaError_t launch_decode_t(const DecodeArgs& a, int grid, cudaStream_t s) {
   constexpr int T = DecodeTraits<E>::kTokensPerStage;
   const DecodeSmem L = decode_smem_layout(a.batch, a.hkv, a.row_bytes, T, G);
-  cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<E, G>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, L.total);
+  // The limit is raised once to the largest layout any batch can need.
+  static int smem_state[kMaxDevicesHost] = {};
+  const int max_bytes = decode_smem_layout(kMaxBatch, 8, 8 * kHeadDim * static_cast<int>(sizeof(E)), T, G).total;
+  if (L.total > max_bytes) return cudaErrorInvalidValue;
+  cudaError_t e = ensure_smem_limit(decode_split_kernel<E, G>, max_bytes, smem_state);
   if (e != cudaSuccess) return e;
   // Both kernels use programmatic dependent launch: the split kernel's set-up
   // (barriers, length scan, first table reads) overlaps the tail of the

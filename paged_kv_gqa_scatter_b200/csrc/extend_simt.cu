@@ -201,8 +201,8 @@ template <typename E, int G>
 cudaError_t launch_t(const ExtendArgs& a, int hkv, int32_t batch, int32_t max_extend, cudaStream_t s) {
   constexpr int QB = kRows / G;
   dim3 grid((max_extend + QB - 1) / QB, hkv, batch);
-  cudaError_t err = cudaFuncSetAttribute(extend_simt_kernel<E, G>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  static int smem_state[kMaxDevicesHost] = {};
+  cudaError_t err = ensure_smem_limit(extend_simt_kernel<E, G>, kSmemBytes, smem_state);
   if (err != cudaSuccess) return err;
   extend_simt_kernel<E, G><<<grid, kThreads, kSmemBytes, s>>>(a);
   return cudaGetLastError();

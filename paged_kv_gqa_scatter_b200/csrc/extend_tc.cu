@@ -656,7 +656,8 @@ cudaError_t launch_g(const CUtensorMap& qm, const ExtendTcArgs& a,
                      int32_t batch, int32_t max_extend, cudaStream_t s) {
   constexpr int TQ = kRowsPerTile / G;
   const int nqb = (max_extend + kQTiles * TQ - 1) / (kQTiles * TQ);
-  cudaError_t e = cudaFuncSetAttribute(extend_tc_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  static int smem_state[kMaxDevicesHost] = {};
+  cudaError_t e = ensure_smem_limit(extend_tc_kernel<G>, kSmemBytes, smem_state);
   if (e != cudaSuccess) return e;
   dim3 grid(nqb, a.hkv, batch);
   extend_tc_kernel<G><<<grid, kThreads, kSmemBytes, s>>>(qm, a);

@@ -10,6 +10,23 @@
 namespace pkv {
 
 constexpr int kHeadDimHost = 128;
+constexpr int kMaxDevicesHost = 64;
+
+// Raise `kernel`'s dynamic shared memory limit to `bytes` once per device.
+// `state` is the caller's per-kernel array (one entry per device) of the
+// limit already set, so calls after the first make no CUDA call at all (this
+// keeps launches legal inside stream capture once the kernel has run once).
+template <typename Kernel>
+inline cudaError_t ensure_smem_limit(Kernel kernel, int bytes, int* state) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevicesHost) return cudaErrorInvalidDevice;
+  if (state[dev] >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) state[dev] = bytes;
+  return e;
+}
 
 struct PoolView {
   const uint8_t* k;  // layer base (bytes)

@@ -1,0 +1,98 @@
+"""store_kv + decode_attn captured in CUDA graphs with fixed buffers (needs a B200).
+
+The serving engine on the pages replays decode from CUDA graphs captured for a
+ladder of batch sizes; a real batch is padded up to the captured size with
+dummy requests whose table row points at a dummy slot and whose context
+length is 1 ("Mini-SGLang 完整剖析", §4.6.6 and §5.3).  Every per-step value the
+kernels read (lengths, table rows, slots, queries) lives in device buffers, so
+one captured graph serves any batch up to its size.  Here each graph is
+replayed twice with different real batches and the real rows are compared
+with the float64 oracle.
+"""
+import numpy as np
+import pytest
+import torch
+
+from gpu_helpers import device_pool, from_dev, i32, oracle_decode, to_dev, tol_check
+from paged_kv_gqa_scatter_b200 import api
+from paged_kv_gqa_scatter_b200 import workloads as W
+
+pytestmark = [pytest.mark.gpu,
+              pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")]
+
+MAX_BS = 256
+LADDER = [1, 8, 64, 256]
+
+
+def test_decode_graph_ladder_with_dummy_padding():
+    rng = np.random.default_rng(77)
+    R = 300
+    lens = rng.integers(1, 700, size=R).astype(np.int32)
+    total = int(lens.sum())
+    # One spare slot beyond the requests' slots becomes the dummy slot.
+    wl = W.decode_small(seq_lens=lens, num_slots=total + 1, num_q_heads=32, num_kv_heads=8, seed=1500)
+    used = set(np.concatenate([wl.page_table[wl.table_idx[r], :lens[r]] for r in range(R)]).tolist())
+    dummy_slot = int(next(s for s in range(wl.pool.num_slots) if s not in used))
+    dummy_row = wl.page_table.shape[0] - 1          # the table's spare last row
+    assert dummy_row not in set(wl.table_idx.tolist())
+    table_np = wl.page_table.copy()
+    table_np[dummy_row, :] = dummy_slot
+    expected, _ = oracle_decode(wl)                 # every request's output after its store
+
+    pool = device_pool(wl.pool, wl.k_planes, wl.v_planes, layers=[0])
+    table = api.PageTable(i32(table_np))
+    Hq, row = wl.num_q_heads, wl.pool.row_elems
+    q_all, k_all, v_all = to_dev(wl.q, W.BF16), to_dev(wl.k_new, W.BF16), to_dev(wl.v_new, W.BF16)
+    loc_all, sl_all, ti_all = i32(wl.out_loc), i32(wl.seq_lens), i32(wl.table_idx)
+
+    # Fixed buffers sized for the largest graph.
+    q = torch.zeros(MAX_BS, Hq, 128, dtype=torch.bfloat16, device="cuda")
+    k_new = torch.zeros(MAX_BS, row, dtype=torch.bfloat16, device="cuda")
+    v_new = torch.zeros_like(k_new)
+    out_loc = torch.full((MAX_BS,), dummy_slot, dtype=torch.int32, device="cuda")
+    seq_lens = torch.ones(MAX_BS, dtype=torch.int32, device="cuda")
+    table_idx = torch.full((MAX_BS,), dummy_row, dtype=torch.int32, device="cuda")
+    out = torch.zeros(MAX_BS, Hq, 128, dtype=torch.bfloat16, device="cuda")
+    ws = api.decode_workspace(MAX_BS, Hq)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+
+    def step(bs):
+        api.store_kv(pool, 0, k_new[:bs], v_new[:bs], out_loc[:bs], err)
+        api.decode_attn(pool, 0, q[:bs], table, table_idx[:bs], seq_lens[:bs], out[:bs], ws,
+                        scale=wl.scale, dev_err=err)
+
+    def load_batch(bs, idx):
+        B = len(idx)
+        ii = torch.as_tensor(idx, dtype=torch.long, device="cuda")
+        q[:B].copy_(q_all[ii]); k_new[:B].copy_(k_all[ii]); v_new[:B].copy_(v_all[ii])
+        out_loc[:B].copy_(loc_all[ii]); seq_lens[:B].copy_(sl_all[ii]); table_idx[:B].copy_(ti_all[ii])
+        q[B:bs].zero_(); k_new[B:bs].zero_(); v_new[B:bs].zero_()
+        out_loc[B:bs].fill_(dummy_slot); seq_lens[B:bs].fill_(1); table_idx[B:bs].fill_(dummy_row)
+
+    # Eager warm-up (first launches happen outside capture), then capture
+    # largest first sharing one memory pool, as the engine on the pages does.
+    for bs in LADDER:
+        load_batch(bs, list(range(min(bs, R))))
+        step(bs)
+    torch.cuda.synchronize()
+    graphs = {}
+    mempool = None
+    s = torch.cuda.Stream()
+    for bs in sorted(LADDER, reverse=True):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, pool=mempool, stream=s):
+            step(bs)
+        mempool = g.pool()
+        graphs[bs] = g
+    torch.cuda.synchronize()
+
+    for bs in LADDER:
+        for B in sorted({bs, max(1, bs // 2 + 1)}):
+            idx = rng.choice(R, size=B, replace=False)
+            load_batch(bs, idx)
+            out.fill_(0)
+            torch.cuda.synchronize()
+            graphs[bs].replay()
+            torch.cuda.synchronize()
+            tol_check(from_dev(out[:B]), expected[idx], W.BF16, f"graph bs={bs} real={B}")
+    assert int(err.item()) == 0
