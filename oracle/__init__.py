@@ -13,12 +13,18 @@ Parity status per function (what pins it, in ``tests/test_oracle_pins.py``):
       returns V, constant K returns mean V, decode == extend with one row,
       q*c with k/c, identical query heads);
   partial_state, combine_states -- merging split states equals the unsplit
-      result.
+      result;
+  rms_norm, rope_rotate_half, qk_norm_rope_store, to_storage -- closed forms
+      (unit-RMS vectors, identity at position 0, a single-pair rotation by a
+      known angle), norm preservation, the relative-position property of
+      rotated dot products, exact bf16 rounding of hand-picked ties.
 The pages print no worked numerical example for any of these, so no stored
 value comes from them.
 """
 from .paged_attention import (attend, combine_states, decode_attn, extend_attn, gather_kv,
                               partial_state, slots_of, store_kv, to_f64)
+from .rope_norm import qk_norm_rope_store, rms_norm, rope_rotate_half, to_storage
 
 __all__ = ["attend", "combine_states", "decode_attn", "extend_attn", "gather_kv",
-           "partial_state", "slots_of", "store_kv", "to_f64"]
+           "partial_state", "qk_norm_rope_store", "rms_norm", "rope_rotate_half", "slots_of",
+           "store_kv", "to_f64", "to_storage"]

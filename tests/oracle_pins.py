@@ -357,3 +357,103 @@ ALL_PINS = [pin_store_bit_copy, pin_page_translation_golden, pin_gather_matches_
             pin_slot_permutation, pin_chunked_equals_unchunked, pin_shared_prefix_equals_private,
             pin_one_token_returns_v, pin_constant_k_mean_v, pin_decode_equals_extend_one_row,
             pin_scale_invariance, pin_identical_heads, pin_split_combine, pin_empty_context_zero]
+
+
+# ---------------------------------------------------------------------------
+# q/k RMSNorm + RoPE + store pins.
+# ---------------------------------------------------------------------------
+def rope_cache(max_pos, d, base=10000.0, dtype=np.float32):
+    """cos | sin halves per position, built here from the angle definition."""
+    half = d // 2
+    inv = base ** (-2.0 * np.arange(half) / d)
+    ang = np.arange(max_pos)[:, None] * inv[None, :]
+    return np.concatenate([np.cos(ang), np.sin(ang)], axis=1).astype(dtype)
+
+
+def pin_bf16_rounding(orc):
+    """Nearest-even rounding to bf16 on hand-picked values and ties."""
+    vals = [1.0, 1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8, 1.0 + 2 ** -8 + 2 ** -40, -2.5, 0.0,
+            3.0 * 2 ** -7, 65280.0, 2.0 ** -100]
+    want = [0x3F80, 0x3F80, 0x3F82, 0x3F81, 0xC020, 0x0000, 0x3CC0, 0x477F, 0x0D80]
+    got = orc.to_storage(np.array(vals), "bf16")
+    assert [int(x) for x in got] == want, [hex(int(x)) for x in got]
+
+
+def pin_rms_norm_closed_form(orc):
+    """A constant vector c has RMS |c|; a 3-4-0 vector has RMS 5/sqrt(d)."""
+    d = D
+    w = np.linspace(0.5, 1.5, d)
+    y = orc.rms_norm(np.full((1, d), -3.0), w, 0.0)
+    _close(y[0], -w, 1e-15)
+    x = np.zeros((1, d)); x[0, 0] = 3.0; x[0, 1] = 4.0
+    y = orc.rms_norm(x, np.ones(d), 0.0)
+    r = 5.0 / math.sqrt(d)
+    _close(y[0, :2], [3.0 / r, 4.0 / r], 1e-15)
+    # eps enters under the root: mean(x^2) = 1, eps = 3 -> scale 1/2.
+    y = orc.rms_norm(np.ones((1, d)), np.ones(d), 3.0)
+    _close(y[0], np.full(d, 0.5), 1e-15)
+
+
+def pin_rope_closed_form(orc):
+    """Position 0 is the identity; a unit vector in dim i turns by angle
+    p * base^(-2i/d) into dim i + d/2."""
+    cache = rope_cache(64, D)
+    rng = np.random.default_rng(61)
+    x = rng.standard_normal((1, 3, D))
+    _close(orc.rope_rotate_half(x, [0], cache), x, 1e-15)
+    for i, p in ((0, 5), (17, 63), (63, 1)):
+        e = np.zeros((1, 1, D)); e[0, 0, i] = 1.0
+        y = orc.rope_rotate_half(e, [p], cache)[0, 0]
+        th = p * 10000.0 ** (-2.0 * i / D)
+        exp = np.zeros(D); exp[i] = math.cos(th); exp[i + D // 2] = math.sin(th)
+        _close(y, exp, 1e-6)   # the cache holds float32 cos/sin
+
+
+def pin_rope_relative_position(orc):
+    """Rotated dot products depend only on the position difference, and the
+    rotation keeps each vector's norm."""
+    cache = rope_cache(256, D, dtype=np.float64)
+    rng = np.random.default_rng(67)
+    q = rng.standard_normal((1, 1, D))
+    k = rng.standard_normal((1, 1, D))
+    ref = None
+    for shift in (0, 7, 100):
+        a = orc.rope_rotate_half(q, [40 + shift], cache)
+        b = orc.rope_rotate_half(k, [13 + shift], cache)
+        dot = float((a * b).sum())
+        ref = dot if ref is None else ref
+        assert abs(dot - ref) < 1e-9 * (1 + abs(ref)), (dot, ref)
+        assert abs(np.linalg.norm(a) - np.linalg.norm(q)) < 1e-9
+
+
+def pin_fused_store(orc):
+    """The fused step returns normed, rotated q; writes rotated k and the
+    untouched v (bit copy) at out_loc; other slots keep their bits."""
+    rng = np.random.default_rng(71)
+    Hq, Hkv, N, S = 4, 2, 3, 16
+    qkv = _bits(_bf16_round(rng.standard_normal((N, (Hq + 2 * Hkv) * D))))
+    pos = np.array([0, 9, 31])
+    cache = rope_cache(32, D)
+    wq = _bf16_round(rng.uniform(0.5, 1.5, D))
+    wk = _bf16_round(rng.uniform(0.5, 1.5, D))
+    kp = {0: rng.integers(0, 1 << 16, (S, Hkv, D), dtype=np.uint16)}
+    vp = {0: rng.integers(0, 1 << 16, (S, Hkv, D), dtype=np.uint16)}
+    k0, v0 = kp[0].copy(), vp[0].copy()
+    loc = np.array([4, 11, 0])
+    q = orc.qk_norm_rope_store(qkv, Hq, Hkv, D, pos, cache, _bits(wq), _bits(wk), 1e-6, kp, vp, 0, loc)
+    x = orc.to_f64(qkv)
+    # position 0 leaves the normed q unrotated
+    q0 = x[0, :Hq * D].reshape(Hq, D)
+    _close(q[0], q0 / np.sqrt((q0 ** 2).mean(axis=1, keepdims=True) + 1e-6) * wq, 1e-12)
+    v_in = qkv[:, (Hq + Hkv) * D:].reshape(N, Hkv, D)
+    for i, sl in enumerate(loc):
+        assert np.array_equal(vp[0][sl], v_in[i])
+    k_first = x[0, Hq * D:(Hq + Hkv) * D].reshape(Hkv, D)
+    kn = k_first / np.sqrt((k_first ** 2).mean(axis=1, keepdims=True) + 1e-6) * wk
+    assert np.array_equal(kp[0][4], _bits(_bf16_round(kn)))
+    rest = np.setdiff1d(np.arange(S), loc)
+    assert np.array_equal(kp[0][rest], k0[rest]) and np.array_equal(vp[0][rest], v0[rest])
+
+
+ALL_PINS += [pin_bf16_rounding, pin_rms_norm_closed_form, pin_rope_closed_form,
+             pin_rope_relative_position, pin_fused_store]

@@ -32,18 +32,45 @@ MUTATIONS = {
     "partial_max_wrong": ("p = np.exp(s - m[h])", "p = np.exp(s)"),
 }
 
+# The same for the q/k norm + RoPE oracle.
+ROPE_MUTATIONS = {
+    "rope_sin_sign": ("x2 * cos + x1 * sin", "x2 * cos - x1 * sin"),
+    "rope_interleaved_pairs": ("x1 = x[..., :half]\n    x2 = x[..., half:]", "x1 = x[..., 0::2]\n    x2 = x[..., 1::2]"),
+    "rms_sum_not_mean": ("ms = np.mean(x * x, axis=-1, keepdims=True)", "ms = np.sum(x * x, axis=-1, keepdims=True)"),
+    "rms_eps_outside": ("return x / np.sqrt(ms + eps) * w", "return x / (np.sqrt(ms) + eps) * w"),
+    "bf16_truncates": ("y = np.ldexp(np.rint(m * 256.0), e - 8)", "y = np.ldexp(np.trunc(m * 256.0), e - 8)"),
+    "v_gets_rotated": ("vl[loc[i]] = to_storage(v[i], storage)", "vl[loc[i]] = to_storage(k[i], storage)"),
+    "k_not_normed": ("k = rope_rotate_half(rms_norm(k, k_norm_w, eps), positions, cos_sin_cache)",
+                     "k = rope_rotate_half(k, positions, cos_sin_cache)"),
+}
+
 
 def _mutant(name):
-    old, new = MUTATIONS[name]
-    src_path = os.path.join(os.path.dirname(oracle.__file__), "paged_attention.py")
-    src = open(src_path).read()
-    assert src.count(old) == 1, f"mutation {name} does not match the oracle source once"
+    """The oracle package with one planted mistake (in either module)."""
+    base = os.path.dirname(oracle.__file__)
+    pa = open(os.path.join(base, "paged_attention.py")).read()
+    rn = open(os.path.join(base, "rope_norm.py")).read()
+    if name in MUTATIONS:
+        old, new = MUTATIONS[name]
+        assert pa.count(old) == 1, f"mutation {name} does not match the oracle source once"
+        pa = pa.replace(old, new)
+    else:
+        old, new = ROPE_MUTATIONS[name]
+        assert rn.count(old) == 1, f"mutation {name} does not match the oracle source once"
+        rn = rn.replace(old, new)
+    m1 = types.ModuleType(f"oracle_pa_{name}")
+    exec(compile(pa, f"<mutant {name} paged_attention>", "exec"), m1.__dict__)
+    m2 = types.ModuleType(f"oracle_rn_{name}")
+    m2.__dict__["to_f64"] = m1.to_f64
+    rn = rn.replace("from .paged_attention import to_f64\n", "")
+    exec(compile(rn, f"<mutant {name} rope_norm>", "exec"), m2.__dict__)
     mod = types.ModuleType(f"oracle_mutant_{name}")
-    exec(compile(src.replace(old, new), f"<mutant {name}>", "exec"), mod.__dict__)
+    for k in oracle.__all__:
+        mod.__dict__[k] = getattr(m1, k) if hasattr(m1, k) else getattr(m2, k)
     return mod
 
 
-@pytest.mark.parametrize("name", sorted(MUTATIONS))
+@pytest.mark.parametrize("name", sorted(MUTATIONS) + sorted(ROPE_MUTATIONS))
 def test_planted_mistake_is_caught(name):
     mod = _mutant(name)
     failed = []
