@@ -66,7 +66,8 @@ typedef enum {
   PKV_DEV_ERR_EMPTY_CONTEXT = 4, /* decode seq_len < 1, or queries with no key          */
   PKV_DEV_ERR_BAD_LENGTH = 8,    /* negative prefix/extend length, or q_offsets broken  */
   PKV_DEV_ERR_PAGE_ALIGN = 16,   /* page_size > 1 and a page's first entry % page_size  */
-  PKV_DEV_ERR_TIMEOUT = 32       /* an internal wait gave up (never expected)           */
+  PKV_DEV_ERR_TIMEOUT = 32,      /* an internal wait gave up (never expected)           */
+  PKV_DEV_ERR_POSITION = 64      /* a RoPE position outside [0, max_position)           */
 } pkv_device_error;
 
 typedef enum { PKV_DTYPE_BF16 = 0, PKV_DTYPE_F32 = 1 } pkv_dtype;
@@ -144,6 +145,44 @@ int pkv_store_kv(const pkv_pool* pool, int32_t layer, const void* k, int64_t k_r
                  const void* v, int64_t v_row_stride, const void* out_loc,
                  int32_t out_loc_is_i64, int64_t n_tokens, int32_t* dev_err,
                  pkv_stream_t stream);
+
+/*
+ * qk_norm_rope_store -- q/k RMSNorm, RoPE and store_kv in one pass over the
+ * rows of the fused qkv projection [P5 §4.6.7: the attention layer splits
+ * qkv, applies q_norm / k_norm per head (Qwen3), rotates q and k in place at
+ * the batch positions, then the backend stores k and v at out_loc; §4.5.6:
+ * one shared RotaryEmbedding holds a cos_sin_cache of max_position x
+ * rotary_dim].
+ *
+ *   for token t < n_tokens, with x = qkv row t = [q heads | k heads | v heads]:
+ *     q_out[t][h]                  = rope(norm(q_h, q_norm_weight), pos[t])
+ *     pool.k[layer][out_loc[t]][g] = rope(norm(k_g, k_norm_weight), pos[t])
+ *     pool.v[layer][out_loc[t]][g] = v_g                      (bit copy)
+ *   norm(x, w) = x / sqrt(mean(x^2) + eps) * w over the 128 dims (skipped
+ *   when the weight pointer is NULL); rope is the rotate-half form over the
+ *   whole head: for i < 64, (x_i, x_{i+64}) -> (x_i c - x_{i+64} s,
+ *   x_{i+64} c + x_i s) with c, s = cos_sin_cache[pos][i], [pos][64 + i].
+ *   The pages do not spell the pairing out; rotate-half is the reading taken.
+ *
+ * qkv: device, pool dtype, rows of (Hq + 2 Hkv) * 128 elements, row stride
+ *   in elements; 16-byte aligned rows.
+ * positions: device int32 (positions_is_i64 = 0) or int64 (= 1) [n_tokens];
+ *   a position outside [0, max_position) zeroes that token's q and k rows and
+ *   sets PKV_DEV_ERR_POSITION.
+ * cos_sin_cache: device float32 [max_position][128] (64 cos then 64 sin),
+ *   16-byte aligned.
+ * q_norm_weight, k_norm_weight: device [128] in the pool dtype, or NULL.
+ * out_loc: as for pkv_store_kv (distinct slots; out of range is skipped and
+ *   flagged).  q_out: device [n_tokens][num_q_heads][128], pool dtype.
+ * All arithmetic is fp32; outputs round to the pool type (nearest even).
+ */
+int pkv_qk_norm_rope_store(const pkv_pool* pool, int32_t layer, const void* qkv,
+                           int64_t qkv_row_stride, int32_t num_q_heads, const void* positions,
+                           int32_t positions_is_i64, const float* cos_sin_cache,
+                           int64_t max_position, const void* q_norm_weight,
+                           const void* k_norm_weight, float eps, const void* out_loc,
+                           int32_t out_loc_is_i64, int64_t n_tokens, void* q_out,
+                           int32_t* dev_err, pkv_stream_t stream);
 
 /*
  * gather_kv -- copies requests' K/V rows, in token order, through the page

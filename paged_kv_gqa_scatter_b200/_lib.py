@@ -36,6 +36,9 @@ SIGNATURES = {
     "pkv_version": (ctypes.c_char_p, []),
     "pkv_store_kv": (ctypes.c_int, [ctypes.POINTER(PkvPool), c_i32, c_vp, c_i64, c_vp, c_i64, c_vp,
                                     c_i32, c_i64, c_vp, c_vp]),
+    "pkv_qk_norm_rope_store": (ctypes.c_int, [ctypes.POINTER(PkvPool), c_i32, c_vp, c_i64, c_i32, c_vp,
+                                              c_i32, c_vp, c_i64, c_vp, c_vp, ctypes.c_float, c_vp,
+                                              c_i32, c_i64, c_vp, c_vp, c_vp]),
     "pkv_gather_kv": (ctypes.c_int, [ctypes.POINTER(PkvPool), c_i32, ctypes.POINTER(PkvPageTable),
                                      c_vp, c_vp, c_vp, c_i32, c_vp, c_vp, c_vp, c_vp]),
     "pkv_decode_workspace_bytes": (c_size, [c_i32, c_i32]),

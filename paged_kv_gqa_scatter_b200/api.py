@@ -18,6 +18,15 @@ from . import _lib
 DTYPE_CODES = {torch.bfloat16: 0, torch.float32: 1}
 HEAD_DIM = 128
 
+# pkv_device_error bits OR-ed into a call's dev_err word.
+DEV_ERR_SLOT_RANGE = 1
+DEV_ERR_TABLE_RANGE = 2
+DEV_ERR_EMPTY_CONTEXT = 4
+DEV_ERR_BAD_LENGTH = 8
+DEV_ERR_PAGE_ALIGN = 16
+DEV_ERR_TIMEOUT = 32
+DEV_ERR_POSITION = 64
+
 
 def _stream_ptr(stream: Optional[torch.cuda.Stream]) -> int:
     s = stream if stream is not None else torch.cuda.current_stream()
@@ -102,6 +111,29 @@ def store_kv(pool: KVPool, layer: int, k: torch.Tensor, v: torch.Tensor, out_loc
                                 v.data_ptr(), v.stride(0), out_loc.data_ptr(),
                                 1 if out_loc.dtype == torch.int64 else 0, out_loc.shape[0],
                                 _ptr(dev_err), _stream_ptr(stream)), "store_kv")
+
+
+def qk_norm_rope_store(pool: KVPool, layer: int, qkv: torch.Tensor, num_q_heads: int,
+                       positions: torch.Tensor, cos_sin_cache: torch.Tensor, out_loc: torch.Tensor,
+                       q_out: torch.Tensor, q_norm_weight: Optional[torch.Tensor] = None,
+                       k_norm_weight: Optional[torch.Tensor] = None, eps: float = 1e-6,
+                       dev_err: Optional[torch.Tensor] = None, stream=None) -> None:
+    """pkv_qk_norm_rope_store: q/k RMSNorm + RoPE, then k/v into the pool, q into q_out."""
+    _require_cuda(qkv, positions, cos_sin_cache, out_loc, q_out, q_norm_weight, k_norm_weight, dev_err)
+    if qkv.dim() != 2 or qkv.dtype != pool.dtype or (qkv.shape[0] > 0 and qkv.stride(1) != 1):
+        raise ValueError("qkv must be [tokens][(Hq + 2 Hkv) * 128] rows of the pool dtype")
+    if cos_sin_cache.dtype != torch.float32 or not cos_sin_cache.is_contiguous():
+        raise ValueError("cos_sin_cache must be contiguous float32 [max_position][128]")
+    for t, name in ((positions, "positions"), (out_loc, "out_loc")):
+        if t.dtype not in (torch.int32, torch.int64) or not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous int32 or int64")
+    lib = _lib.load()
+    _lib.check(lib.pkv_qk_norm_rope_store(
+        ctypes.byref(pool.c), layer, qkv.data_ptr(), qkv.stride(0), num_q_heads,
+        positions.data_ptr(), 1 if positions.dtype == torch.int64 else 0, cos_sin_cache.data_ptr(),
+        cos_sin_cache.shape[0], _ptr(q_norm_weight), _ptr(k_norm_weight), float(eps),
+        out_loc.data_ptr(), 1 if out_loc.dtype == torch.int64 else 0, qkv.shape[0],
+        q_out.data_ptr(), _ptr(dev_err), _stream_ptr(stream)), "qk_norm_rope_store")
 
 
 def gather_kv(pool: KVPool, layer: int, table: PageTable, table_idx: torch.Tensor,

@@ -115,6 +115,35 @@ int pkv_store_kv(const pkv_pool* pool, int32_t layer, const void* k, int64_t k_r
                                         static_cast<cudaStream_t>(stream)));
 }
 
+int pkv_qk_norm_rope_store(const pkv_pool* pool, int32_t layer, const void* qkv,
+                           int64_t qkv_row_stride, int32_t num_q_heads, const void* positions,
+                           int32_t positions_is_i64, const float* cos_sin_cache,
+                           int64_t max_position, const void* q_norm_weight,
+                           const void* k_norm_weight, float eps, const void* out_loc,
+                           int32_t out_loc_is_i64, int64_t n_tokens, void* q_out,
+                           int32_t* dev_err, pkv_stream_t stream) {
+  PoolView pv;
+  int st = check_pool(pool, layer, &pv);
+  if (st != PKV_OK) return st;
+  if (n_tokens < 0 || max_position < 1) return PKV_ERR_INVALID_ARG;
+  if (n_tokens == 0) return PKV_OK;
+  if (num_q_heads < 1) return PKV_ERR_INVALID_ARG;
+  if (!qkv || !positions || !cos_sin_cache || !out_loc || !q_out) return PKV_ERR_INVALID_ARG;
+  if (positions_is_i64 != 0 && positions_is_i64 != 1) return PKV_ERR_INVALID_ARG;
+  if (out_loc_is_i64 != 0 && out_loc_is_i64 != 1) return PKV_ERR_INVALID_ARG;
+  if (!(eps >= 0.f)) return PKV_ERR_INVALID_ARG;
+  const int64_t row = static_cast<int64_t>(num_q_heads + 2 * pool->num_kv_heads) * pool->head_dim;
+  if (qkv_row_stride < row) return PKV_ERR_INVALID_ARG;
+  if (!aligned16(qkv) || (qkv_row_stride * pv.esize) % 16 != 0 || !aligned16(q_out) ||
+      !aligned16(cos_sin_cache) || (q_norm_weight && !aligned16(q_norm_weight)) ||
+      (k_norm_weight && !aligned16(k_norm_weight)))
+    return PKV_ERR_MISALIGNED;
+  return from_cuda(pkv::launch_qk_norm_rope_store(
+      pv, qkv, qkv_row_stride, num_q_heads, positions, positions_is_i64 == 1, cos_sin_cache,
+      max_position, q_norm_weight, k_norm_weight, eps, out_loc, out_loc_is_i64 == 1, n_tokens,
+      q_out, dev_err, static_cast<cudaStream_t>(stream)));
+}
+
 int pkv_gather_kv(const pkv_pool* pool, int32_t layer, const pkv_page_table* table,
                   const int32_t* table_idx, const int32_t* seq_lens, const int64_t* row_offsets,
                   int32_t batch, void* k_out, void* v_out, int32_t* dev_err,

@@ -52,6 +52,12 @@ cudaError_t launch_store_kv(const PoolView& pool, const void* k, int64_t k_strid
                             const void* v, int64_t v_stride_bytes, const void* out_loc,
                             bool loc_i64, int64_t n, int32_t* err, cudaStream_t s);
 
+cudaError_t launch_qk_norm_rope_store(const PoolView& pool, const void* qkv, int64_t qkv_row_stride,
+                                      int32_t num_q_heads, const void* positions, bool pos_i64,
+                                      const float* cos_sin, int64_t max_position, const void* q_w,
+                                      const void* k_w, float eps, const void* out_loc, bool loc_i64,
+                                      int64_t n, void* q_out, int32_t* err, cudaStream_t s);
+
 cudaError_t launch_gather_kv(const PoolView& pool, const TableView& t, const int32_t* table_idx,
                              const int32_t* seq_lens, const int64_t* row_offsets, int32_t batch,
                              void* k_out, void* v_out, int32_t* err, cudaStream_t s);

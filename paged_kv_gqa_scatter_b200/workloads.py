@@ -572,3 +572,69 @@ def decode_paged_small(dtype: str = BF16, seq_lens=(1, 16, 17, 300, 1029), page_
     out_loc = np.array([table[table_idx[r], seq_lens[r] - 1] for r in range(B)], dtype=np.int32)
     return DecodeWorkload("decode-paged-small", spec, num_q_heads, 0, kp, vp, table, table_idx,
                           seq_lens, q, k_new, v_new, out_loc, 1.0 / math.sqrt(HEAD_DIM))
+
+
+# ---------------------------------------------------------------------------
+# The step ahead of attention: q/k norm + RoPE + store, on a fused qkv output.
+# ---------------------------------------------------------------------------
+@dataclasses.dataclass
+class RopeStoreWorkload:
+    """One layer's qkv rows for N tokens, their positions and slots."""
+    name: str
+    pool: PoolSpec
+    num_q_heads: int
+    layer: int
+    k_planes: Dict[int, np.ndarray]
+    v_planes: Dict[int, np.ndarray]
+    qkv: np.ndarray            # [N][(Hq + 2 Hkv) * d]
+    positions: np.ndarray      # int32 [N]
+    cos_sin_cache: np.ndarray  # float32 [max_position][d]: cos halves, then sin halves
+    q_norm_w: Optional[np.ndarray]  # [d] or None
+    k_norm_w: Optional[np.ndarray]
+    eps: float
+    out_loc: np.ndarray        # int32 [N]
+
+    @property
+    def n_tokens(self) -> int:
+        return int(self.qkv.shape[0])
+
+
+def rotary_table(max_position: int, head_dim: int = HEAD_DIM, base: float = 1e6) -> np.ndarray:
+    """The RotaryEmbedding input table: row p holds cos(p * base^(-2i/d)) for
+    i < d/2, then the sines of the same angles, as float32.  It is a model
+    constant handed to both sides, like a weight."""
+    half = head_dim // 2
+    inv = base ** (-(2.0 * np.arange(half, dtype=np.float64)) / head_dim)
+    ang = np.arange(max_position, dtype=np.float64)[:, None] * inv[None, :]
+    return np.concatenate([np.cos(ang), np.sin(ang)], axis=1).astype(np.float32)
+
+
+def rope_store_step(dtype: str = BF16, positions=None, num_q_heads: int = 16,
+                    num_kv_heads: int = 8, num_slots: int = 4096, max_position: int = 8192,
+                    norms: bool = True, seed: Optional[int] = None, x_scale: float = 2.0,
+                    name: str = "rope-store") -> RopeStoreWorkload:
+    """N tokens of a Qwen3-style layer: qkv rows N(0, x_scale^2), norm weights
+    1 + N(0, 0.1^2) (learned scales near one), positions as given (default 45
+    tokens spread over [0, max_position)), distinct random slots of a
+    single-layer pool whose other slots hold random rows."""
+    rng = np.random.Generator(np.random.PCG64(seed_for(6) if seed is None else seed))
+    if positions is None:
+        positions = rng.integers(0, max_position, size=45)
+    positions = np.asarray(positions, dtype=np.int32)
+    n = positions.shape[0]
+    spec = PoolSpec(1, num_slots, num_kv_heads, HEAD_DIM, 1, dtype)
+    kp = _new_plane_dict(spec, [0])
+    vp = _new_plane_dict(spec, [0])
+    all_slots = np.arange(num_slots)
+    _fill_slots(rng, kp[0], all_slots, dtype)
+    _fill_slots(rng, vp[0], all_slots, dtype)
+    row = (num_q_heads + 2 * num_kv_heads) * HEAD_DIM
+    qkv = draw_values(rng, (n, row), dtype, x_scale)
+    qw = kw = None
+    if norms:
+        w = 1.0 + 0.1 * rng.standard_normal(size=(2, HEAD_DIM)).astype(np.float32)
+        qw = f32_to_bf16_bits(w[0]) if dtype == BF16 else w[0].copy()
+        kw = f32_to_bf16_bits(w[1]) if dtype == BF16 else w[1].copy()
+    out_loc = rng.choice(num_slots, size=n, replace=False).astype(np.int32)
+    return RopeStoreWorkload(name, spec, num_q_heads, 0, kp, vp, qkv, positions,
+                             rotary_table(max_position), qw, kw, 1e-6, out_loc)
