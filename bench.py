@@ -441,7 +441,68 @@ def run_decode(args, world, rank, local):
                                   "kind": "oracle", "sample": sample}
     if not args.no_extend and args.workload == "decode-qwen3-0.6b":
         result["extend"] = run_extend_measure(dev, warmup=3, iters=max(5, args.steps))
+        result["qk_norm_rope_store"] = run_rope_measure(dev, iters=max(5, args.steps))
     return result
+
+
+def rope_bytes(n: int, hq: int, hkv: int, esize: int = 2) -> int:
+    """Algorithmic bytes of one fused q/k norm + RoPE + store call: each token's
+    qkv row read, its q row and its k and v rows written, its position, slot
+    and cos/sin row read (the norm weights are negligible)."""
+    row = (hq + 2 * hkv) * 128 * esize
+    return n * (2 * row + 4 + 4 + 128 * 4)
+
+
+def run_rope_measure(dev, iters=10, warmup=3):
+    """The fused q/k norm + RoPE + store call on three shapes: this decode
+    step's 64 tokens (Hq 16, Hkv 8), and 2048- and 16384-token prefill batches
+    of the Qwen3-8B shape (Hq 32, Hkv 8).  L2 is flushed before every timed call."""
+    import torch
+    from paged_kv_gqa_scatter_b200 import api
+    from paged_kv_gqa_scatter_b200 import workloads as W
+    hbm, _, _, src = measured_peaks()
+    # L2 flush by reading a 256 MB buffer: it leaves clean lines, so the timed
+    # call does not pay for writing back a flush buffer's dirty ones.
+    flush = torch.ones(64 << 20, dtype=torch.int32, device=dev)
+    cache = torch.from_numpy(W.rotary_table(40960)).to(dev)
+    g = torch.Generator(device=dev)
+    g.manual_seed(6)
+    out = {}
+    for name, n, hq, hkv in (("decode batch 64, Hq 16 Hkv 8", 64, 16, 8),
+                             ("prefill chunk 2048, Hq 32 Hkv 8", 2048, 32, 8),
+                             ("prefill batch 16384, Hq 32 Hkv 8", 16384, 32, 8)):
+        row = (hq + 2 * hkv) * 128
+        qkv = torch.randn(n, row, device=dev, generator=g).to(torch.bfloat16)
+        slots = 4 * n
+        pool = api.KVPool.empty(1, slots, hkv, device=dev)
+        pos = torch.randint(0, 40960, (n,), device=dev, dtype=torch.int32, generator=g)
+        loc = torch.randperm(slots, device=dev, generator=g)[:n].to(torch.int32)
+        w = (1.0 + 0.1 * torch.randn(2, 128, device=dev, generator=g)).to(torch.bfloat16)
+        q_out = torch.empty(n, hq, 128, device=dev, dtype=torch.bfloat16)
+        err = torch.zeros(1, dtype=torch.int32, device=dev)
+
+        def call():
+            api.qk_norm_rope_store(pool, 0, qkv, hq, pos, cache, loc, q_out, w[0], w[1], 1e-6, err)
+        for _ in range(warmup):
+            call()
+        s = torch.cuda.current_stream(dev)
+        ts = []
+        for _ in range(iters):
+            flush.sum()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(s)
+            call()
+            b.record(s)
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b))
+        ts.sort()
+        us = ts[len(ts) // 2] * 1e3
+        nbytes = rope_bytes(n, hq, hkv)
+        gbs = nbytes / us / 1e3
+        out[name] = {"us": round(us, 3), "bytes": nbytes, "GB/s": round(gbs, 1),
+                     "frac": round(gbs / hbm, 4), "peak": hbm, "peak_source": src,
+                     "device_error_word": int(err.item())}
+    return out
 
 
 def run_extend_measure(dev, warmup=3, iters=10):
