@@ -266,6 +266,45 @@ int pkv_decode_attn_noalloc(const pkv_pool* pool, int32_t layer, const void* q,
                             float scale, void* out, int32_t* dev_err, pkv_stream_t stream);
 
 /*
+ * decode_attn_cascade -- decode_attn for batches whose requests share
+ * radix-cached prefixes [P5 §1.4: requests with a common prefix point their
+ * table rows at the same slots; §1.2: decode is memory bound].
+ *
+ *   The result is decode_attn's: out[r][h] = attention of q[r][h] over the
+ *   first seq_lens[r] tokens of row table_idx[r].  The requests form
+ *   num_groups contiguous groups, group g = requests group_offsets[g] ..
+ *   group_offsets[g+1] - 1, whose first group_prefix_lens[g] context tokens
+ *   are the same slots (the caller's promise: the call reads them from the
+ *   row of the group's first request only).
+ *
+ * The shared prefix is attended once per group with all members' query rows
+ * stacked on the tcgen05 tensor cores (its K/V are read once per group, not
+ * once per request); each request's own suffix goes through the split-KV
+ * decode kernel; the partial results are merged by their (max, sum) pairs.
+ * This is not on the pages; it is the reuse their prefix sharing allows.
+ *
+ * group_offsets: device int32 [num_groups + 1], 0 = first <= ... <= last =
+ *   batch.  group_prefix_lens: device int32 [num_groups], each 0 <= p_g <=
+ *   min over members of seq_lens and <= max_prefix_len (host int64, sizes
+ *   the prefix pass and the workspace; <= table cols).  A violation sets
+ *   PKV_DEV_ERR_BAD_LENGTH and the affected results are unspecified but
+ *   finite.
+ * workspace: pkv_decode_cascade_workspace_bytes(batch, num_q_heads,
+ *   max_prefix_len) bytes, 16-byte aligned.
+ * bf16 pools only (PKV_ERR_UNSUPPORTED otherwise); other limits as
+ * decode_attn.
+ */
+size_t pkv_decode_cascade_workspace_bytes(int32_t batch, int32_t num_q_heads,
+                                          int64_t max_prefix_len);
+int pkv_decode_attn_cascade(const pkv_pool* pool, int32_t layer, const void* q,
+                            int32_t num_q_heads, const pkv_page_table* table,
+                            const int32_t* table_idx, const int32_t* seq_lens, int32_t batch,
+                            const int32_t* group_offsets, const int32_t* group_prefix_lens,
+                            int32_t num_groups, int64_t max_prefix_len, float scale, void* out,
+                            void* workspace, size_t workspace_bytes, int32_t* dev_err,
+                            pkv_stream_t stream);
+
+/*
  * extend_attn [P4 chunked prefill: every chunk of a request uses the same
  * table row and reuses the KV of the chunks before it; P5 §4.2.3: a request
  * has cached_len (its prefix, possibly radix-shared) and extend_len =

@@ -46,6 +46,11 @@ SIGNATURES = {
                                        ctypes.POINTER(PkvPageTable), c_vp, c_vp, c_i32,
                                        ctypes.c_float, c_vp, c_vp, c_size, c_vp, c_vp]),
     "pkv_decode_noalloc_max_scratch_bytes": (c_size, []),
+    "pkv_decode_cascade_workspace_bytes": (c_size, [c_i32, c_i32, c_i64]),
+    "pkv_decode_attn_cascade": (ctypes.c_int, [ctypes.POINTER(PkvPool), c_i32, c_vp, c_i32,
+                                               ctypes.POINTER(PkvPageTable), c_vp, c_vp, c_i32,
+                                               c_vp, c_vp, c_i32, c_i64, ctypes.c_float, c_vp,
+                                               c_vp, c_size, c_vp, c_vp]),
     "pkv_decode_attn_noalloc": (ctypes.c_int, [ctypes.POINTER(PkvPool), c_i32, c_vp, c_i32,
                                                ctypes.POINTER(PkvPageTable), c_vp, c_vp, c_i32,
                                                ctypes.c_float, c_vp, c_vp, c_vp]),

@@ -200,6 +200,43 @@ def decode_attn_noalloc(pool: KVPool, layer: int, q: torch.Tensor, table: PageTa
                                            _ptr(dev_err), _stream_ptr(stream)), "decode_attn_noalloc")
 
 
+def decode_cascade_workspace_bytes(batch: int, num_q_heads: int, max_prefix_len: int) -> int:
+    return int(_lib.load().pkv_decode_cascade_workspace_bytes(batch, num_q_heads, max_prefix_len))
+
+
+def decode_cascade_workspace(batch: int, num_q_heads: int, max_prefix_len: int,
+                             device="cuda") -> torch.Tensor:
+    n = decode_cascade_workspace_bytes(batch, num_q_heads, max_prefix_len)
+    return torch.empty(max(n, 16), dtype=torch.uint8, device=device)
+
+
+def decode_attn_cascade(pool: KVPool, layer: int, q: torch.Tensor, table: PageTable,
+                        table_idx: torch.Tensor, seq_lens: torch.Tensor,
+                        group_offsets: torch.Tensor, group_prefix_lens: torch.Tensor,
+                        max_prefix_len: int, out: torch.Tensor, workspace: torch.Tensor,
+                        scale: Optional[float] = None, dev_err: Optional[torch.Tensor] = None,
+                        stream=None) -> None:
+    """pkv_decode_attn_cascade: decode_attn with each group's shared prefix
+    attended once per group (tensor cores) and merged with the suffixes."""
+    _require_cuda(q, table_idx, seq_lens, group_offsets, group_prefix_lens, out, workspace, dev_err)
+    if not (q.is_contiguous() and out.is_contiguous()):
+        raise ValueError("q and out must be contiguous")
+    if q.dtype != pool.dtype or out.dtype != pool.dtype:
+        raise ValueError("q/out dtype must match the pool")
+    for t, name in ((group_offsets, "group_offsets"), (group_prefix_lens, "group_prefix_lens")):
+        if t.dtype != torch.int32 or not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous int32")
+    B, Hq, D = q.shape
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    lib = _lib.load()
+    _lib.check(lib.pkv_decode_attn_cascade(
+        ctypes.byref(pool.c), layer, q.data_ptr(), Hq, ctypes.byref(table.c), table_idx.data_ptr(),
+        seq_lens.data_ptr(), B, group_offsets.data_ptr(), group_prefix_lens.data_ptr(),
+        group_prefix_lens.numel(), int(max_prefix_len), scale, out.data_ptr(), workspace.data_ptr(),
+        workspace.numel() * workspace.element_size(), _ptr(dev_err), _stream_ptr(stream)),
+        "decode_attn_cascade")
+
+
 def extend_workspace_bytes(batch: int, num_q_heads: int, total_q: int) -> int:
     return int(_lib.load().pkv_extend_workspace_bytes(batch, num_q_heads, total_q))
 

@@ -195,6 +195,44 @@ int pkv_decode_attn(const pkv_pool* pool, int32_t layer, const void* q, int32_t 
                                       static_cast<cudaStream_t>(stream)));
 }
 
+size_t pkv_decode_cascade_workspace_bytes(int32_t batch, int32_t num_q_heads,
+                                          int64_t max_prefix_len) {
+  if (batch < 0 || num_q_heads < 1 || max_prefix_len < 0) return 0;
+  return pkv::cascade_workspace_bytes(batch, num_q_heads, max_prefix_len);
+}
+
+int pkv_decode_attn_cascade(const pkv_pool* pool, int32_t layer, const void* q,
+                            int32_t num_q_heads, const pkv_page_table* table,
+                            const int32_t* table_idx, const int32_t* seq_lens, int32_t batch,
+                            const int32_t* group_offsets, const int32_t* group_prefix_lens,
+                            int32_t num_groups, int64_t max_prefix_len, float scale, void* out,
+                            void* workspace, size_t workspace_bytes, int32_t* dev_err,
+                            pkv_stream_t stream) {
+  PoolView pv;
+  TableView tv;
+  int st = check_pool(pool, layer, &pv);
+  if (st != PKV_OK) return st;
+  if (pv.dtype != PKV_DTYPE_BF16) return PKV_ERR_UNSUPPORTED;
+  st = check_heads(pool, num_q_heads);
+  if (st != PKV_OK) return st;
+  if (batch < 0 || num_groups < 0 || max_prefix_len < 0) return PKV_ERR_INVALID_ARG;
+  if (batch == 0) return PKV_OK;
+  if (num_groups < 1 || num_groups > batch) return PKV_ERR_INVALID_ARG;
+  if (batch > kMaxDecodeBatch) return PKV_ERR_TOO_LARGE;
+  st = check_table(table, &tv);
+  if (st != PKV_OK) return st;
+  if (static_cast<int64_t>(batch) * tv.cols > INT_MAX || max_prefix_len > tv.cols) return PKV_ERR_TOO_LARGE;
+  if (!q || !out || !table_idx || !seq_lens || !group_offsets || !group_prefix_lens)
+    return PKV_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(out)) return PKV_ERR_MISALIGNED;
+  const size_t need = pkv::cascade_workspace_bytes(batch, num_q_heads, max_prefix_len);
+  if (workspace == nullptr || workspace_bytes < need || !aligned16(workspace)) return PKV_ERR_WORKSPACE;
+  return from_cuda(pkv::launch_decode_cascade(pv, tv, q, num_q_heads, table_idx, seq_lens, batch,
+                                              group_offsets, group_prefix_lens, num_groups,
+                                              max_prefix_len, scale, out, workspace, dev_err,
+                                              static_cast<cudaStream_t>(stream)));
+}
+
 size_t pkv_extend_workspace_bytes(int32_t batch, int32_t num_q_heads, int64_t total_q) {
   (void)batch;
   (void)num_q_heads;

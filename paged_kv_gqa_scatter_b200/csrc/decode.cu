@@ -75,6 +75,11 @@ struct DecodeArgs {
   float2* ws_ml;      // [(grid + batch) * hq]
   float* ws_o;        // [(grid + batch) * hq * 128]
   int32_t* err;
+  // Cascade suffix pass: request r reads context columns kv_start[r] ..
+  // seq_lens[r] - 1 only, and every piece writes a partial (the combine
+  // kernel merges them with the shared-prefix partials).
+  const int32_t* kv_start;  // [batch] or null
+  int32_t cascade;
 };
 
 // Shared memory layout (bytes), identical on host and device.
@@ -174,6 +179,10 @@ __global__ void __launch_bounds__(32 * 9, 1) decode_split_kernel(const DecodeArg
         if (n > a.table_cols) set_err(a.err, PKV_DEV_ERR_TABLE_RANGE);
       }
       n = n < 0 ? 0 : (n > a.table_cols ? static_cast<int32_t>(a.table_cols) : n);
+      if (a.kv_start != nullptr) {  // columns before kv_start[r] are not this pass's
+        const int32_t st = a.kv_start[r];
+        n = st <= 0 ? n : (st >= n ? 0 : n - st);
+      }
       cum[r + 1] = n;
       ssum += n;
     }
@@ -219,7 +228,8 @@ __global__ void __launch_bounds__(32 * 9, 1) decode_split_kernel(const DecodeArg
     const uint64_t policy = policy_evict_first();
     struct Cursor {
       int r;
-      int64_t j0, jb;
+      int64_t j0, jb;  // piece tokens [j0, jb) of the pass, relative to col0
+      int32_t col0;    // table column of the pass's token 0
       const int32_t* rowp;
       bool row_ok;
     };
@@ -233,6 +243,7 @@ __global__ void __launch_bounds__(32 * 9, 1) decode_split_kernel(const DecodeArg
           c.row_ok = trow >= 0 && trow < a.table_rows;
           if (!c.row_ok && lane == 0) set_err(a.err, PKV_DEV_ERR_TABLE_RANGE);
           c.rowp = a.table + (c.row_ok ? trow : 0) * a.table_stride;
+          c.col0 = a.kv_start != nullptr ? max(a.kv_start[rr], 0) : 0;
           c.r = rr;
           c.j0 = ja;
           c.jb = jb;
@@ -252,7 +263,7 @@ __global__ void __launch_bounds__(32 * 9, 1) decode_split_kernel(const DecodeArg
     auto lookup = [&](const Cursor& c, bool have) -> int32_t {
       const int64_t j = c.j0 + lane;
       if (!have || lane >= T || j >= c.jb || !c.row_ok) return 0;
-      const int32_t j32 = static_cast<int32_t>(j);
+      const int32_t j32 = c.col0 + static_cast<int32_t>(j);
       return a.page_size == 1 ? c.rowp[j32] : c.rowp[j32 - page_offset(j32, a.page_size)];
     };
     Cursor c0{}, c1{}, c2{};
@@ -292,7 +303,7 @@ __global__ void __launch_bounds__(32 * 9, 1) decode_split_kernel(const DecodeArg
         if (a.page_size == 1) {
           slot = e0;
         } else if (page_offset(e0, a.page_size) == 0) {
-          slot = static_cast<int64_t>(e0) + page_offset(static_cast<int32_t>(j), a.page_size);
+          slot = static_cast<int64_t>(e0) + page_offset(c0.col0 + static_cast<int32_t>(j), a.page_size);
         } else {
           aligned = false;
           set_err(a.err, PKV_DEV_ERR_PAGE_ALIGN);
@@ -353,7 +364,7 @@ __global__ void __launch_bounds__(32 * 9, 1) decode_split_kernel(const DecodeArg
     const int64_t ja = max(lo, (int64_t)cum[r]) - cum[r];
     const int64_t jb = min(hi, (int64_t)cum[r + 1]) - cum[r];
     if (jb <= ja) continue;
-    const bool whole = cum[r] >= lo && cum[r + 1] <= hi;
+    const bool whole = !a.cascade && cum[r] >= lo && cum[r + 1] <= hi;
     // Warm L2 with the next request's queries while this piece runs.
     if (r + 1 < B && cum[r + 1] < hi && lane < 2 * G)
       asm volatile("prefetch.global.L2 [%0];" ::"l"(qbase + ((int64_t)(r + 1) * a.hq + g * G) * kHeadDim +
@@ -519,11 +530,17 @@ __global__ void __launch_bounds__(32 * 9, 1) decode_split_kernel(const DecodeArg
 // of empty contexts.  One warp per (request, q head); lane owns 4 dims.  The
 // pieces' (max, sum) pairs are read in parallel across lanes and the partial
 // rows with independent loads, so the merge costs a few memory round trips.
+//
+// Cascade mode (pre_ml != null): every request also has nsplit shared-prefix
+// partials, [split][request][head], merged first; partials with sum 0 (empty
+// ranges) are skipped, and the suffix pieces are merged even when there is
+// only one.
 template <typename E>
 __global__ void __launch_bounds__(128) decode_combine_kernel(
     const int32_t* __restrict__ seq_lens, const int32_t* __restrict__ cum,
     const int64_t* __restrict__ per_p, const float2* __restrict__ ml, const float* __restrict__ o,
-    int32_t hq, void* __restrict__ out) {
+    int32_t hq, void* __restrict__ out, const float2* __restrict__ pre_ml,
+    const float* __restrict__ pre_o, int32_t nsplit) {
   // Partials come from the split kernel launched just before this one.
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const int r = blockIdx.x;
@@ -532,7 +549,8 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(
   if (h >= hq) return;
   E* dst = static_cast<E*>(out) + ((int64_t)r * hq + h) * kHeadDim + 4 * lane;
   const int64_t c0 = cum[r], c1 = cum[r + 1];
-  if (seq_lens[r] < 1 || c1 <= c0) {
+  const bool cascade = pre_ml != nullptr;
+  if (seq_lens[r] < 1 || (c1 <= c0 && !cascade)) {
     if constexpr (sizeof(E) == 2) {
       *reinterpret_cast<uint2*>(dst) = make_uint2(0, 0);
     } else {
@@ -541,16 +559,15 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(
     return;
   }
   const int64_t per = *per_p;
-  const int64_t k_lo = c0 / per, k_hi = (c1 - 1) / per;
-  if (k_lo == k_hi) return;  // written by its only piece
+  const int64_t k_lo = c1 > c0 ? c0 / per : 0, k_hi = c1 > c0 ? (c1 - 1) / per : -1;
+  if (!cascade && k_lo == k_hi) return;  // written by its only piece
   // Online merge: the loads of consecutive pieces are independent, so the
-  // unrolled loop keeps several in flight.
+  // unrolled loops keep several in flight.
   float M = -INFINITY, den = 0.f;
   float4 acc = make_float4(0, 0, 0, 0);
-#pragma unroll 4
-  for (int64_t k = k_lo; k <= k_hi; ++k) {
-    const float2 st = ml[(k + r) * hq + h];
-    const float4 x = *reinterpret_cast<const float4*>(o + ((k + r) * hq + h) * kHeadDim + 4 * lane);
+  auto merge = [&](float2 st, const float* src) {
+    if (!(st.y > 0.f)) return;  // empty partial
+    const float4 x = *reinterpret_cast<const float4*>(src + 4 * lane);
     const float Mn = fmaxf(M, st.x);
     const float wa = exp2f(M - Mn), wb = exp2f(st.x - Mn);
     den = den * wa + wb * st.y;
@@ -559,7 +576,15 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(
     acc.z = acc.z * wa + wb * x.z;
     acc.w = acc.w * wa + wb * x.w;
     M = Mn;
+  };
+  const int64_t B = gridDim.x;
+#pragma unroll 4
+  for (int sp = 0; sp < nsplit; ++sp) {
+    const int64_t id = (sp * B + r) * hq + h;
+    merge(pre_ml[id], pre_o + id * kHeadDim);
   }
+#pragma unroll 4
+  for (int64_t k = k_lo; k <= k_hi; ++k) merge(ml[(k + r) * hq + h], o + ((k + r) * hq + h) * kHeadDim);
   const float inv = den > 0.f ? 1.f / den : 0.f;
   if constexpr (sizeof(E) == 2) {
     uint2 w;
@@ -572,7 +597,7 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(
 }
 
 template <typename E, int G>
-cudaError_t launch_decode_t(const DecodeArgs& a, int grid, cudaStream_t s) {
+cudaError_t launch_decode_t(const DecodeArgs& a, int grid, cudaStream_t s, const CascadeView* cv) {
   constexpr int T = DecodeTraits<E>::kTokensPerStage;
   const DecodeSmem L = decode_smem_layout(a.batch, a.hkv, a.row_bytes, T, G);
   // The limit is raised once to the largest layout any batch can need.
@@ -604,7 +629,8 @@ cudaError_t launch_decode_t(const DecodeArgs& a, int grid, cudaStream_t s) {
   ccfg.dynamicSmemBytes = 0;
   return cudaLaunchKernelEx(&ccfg, decode_combine_kernel<E>, a.seq_lens, (const int32_t*)a.ws_cum,
                             (const int64_t*)a.ws_per, (const float2*)a.ws_ml, (const float*)a.ws_o,
-                            a.hq, a.out);
+                            a.hq, a.out, cv ? cv->pre_ml : nullptr, cv ? cv->pre_o : nullptr,
+                            cv ? cv->nsplit : 0);
 }
 
 }  // namespace
@@ -630,7 +656,7 @@ size_t decode_workspace_bytes(int32_t batch, int32_t num_q_heads, int grid) {
 cudaError_t launch_decode(const PoolView& pool, const TableView& t, const void* q,
                           int32_t num_q_heads, const int32_t* table_idx, const int32_t* seq_lens,
                           int32_t batch, float scale, void* out, void* workspace, int grid,
-                          int32_t* err, cudaStream_t s) {
+                          int32_t* err, cudaStream_t s, const CascadeView* cascade) {
   if (batch == 0) return cudaSuccess;
   DecodeArgs a;
   a.kbase = pool.k;
@@ -662,20 +688,22 @@ cudaError_t launch_decode(const PoolView& pool, const TableView& t, const void* 
   w = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(w) + 15) & ~uintptr_t(15));
   a.ws_o = reinterpret_cast<float*>(w);
   a.err = err;
+  a.kv_start = cascade ? cascade->kv_start : nullptr;
+  a.cascade = cascade ? 1 : 0;
   const int G = num_q_heads / pool.num_kv_heads;
   if (pool.dtype == PKV_DTYPE_BF16) {
     switch (G) {
-      case 1: return launch_decode_t<__nv_bfloat16, 1>(a, grid, s);
-      case 2: return launch_decode_t<__nv_bfloat16, 2>(a, grid, s);
-      case 4: return launch_decode_t<__nv_bfloat16, 4>(a, grid, s);
-      case 8: return launch_decode_t<__nv_bfloat16, 8>(a, grid, s);
+      case 1: return launch_decode_t<__nv_bfloat16, 1>(a, grid, s, cascade);
+      case 2: return launch_decode_t<__nv_bfloat16, 2>(a, grid, s, cascade);
+      case 4: return launch_decode_t<__nv_bfloat16, 4>(a, grid, s, cascade);
+      case 8: return launch_decode_t<__nv_bfloat16, 8>(a, grid, s, cascade);
     }
   } else {
     switch (G) {
-      case 1: return launch_decode_t<float, 1>(a, grid, s);
-      case 2: return launch_decode_t<float, 2>(a, grid, s);
-      case 4: return launch_decode_t<float, 4>(a, grid, s);
-      case 8: return launch_decode_t<float, 8>(a, grid, s);
+      case 1: return launch_decode_t<float, 1>(a, grid, s, cascade);
+      case 2: return launch_decode_t<float, 2>(a, grid, s, cascade);
+      case 4: return launch_decode_t<float, 4>(a, grid, s, cascade);
+      case 8: return launch_decode_t<float, 8>(a, grid, s, cascade);
     }
   }
   return cudaErrorInvalidValue;

@@ -109,6 +109,18 @@ struct ExtendTcArgs {
   int32_t hq, hkv;
   float scale_log2;
   int32_t* err;
+  // Prefix mode (the shared-prefix pass of cascade decode).  blockIdx.z =
+  // group * nsplit + split; q_offsets are the group offsets, prefix_lens the
+  // groups' shared prefix lengths.  Every query row of group g (one decode
+  // token per member request, no causal mask) attends to keys
+  // [split * split_keys, min(p_g, (split + 1) * split_keys)) of the group
+  // leader's table row and writes an un-normalised fp32 partial plus its
+  // (max, sum) instead of bf16 output.
+  int32_t prefix_mode;
+  int32_t nsplit, split_keys;
+  int32_t nreq;    // query rows (requests) in q
+  float2* pre_ml;  // [nsplit][nreq][hq]
+  float* pre_o;    // [nsplit][nreq][hq][128]
 };
 
 // ---- PTX wrappers -----------------------------------------------------------
@@ -268,12 +280,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int32_t* abort_flag = reinterpret_cast<volatile int32_t*>(smem + kOffMisc + 16);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int r = blockIdx.z, g = blockIdx.y;
+  const int g = blockIdx.y;
+  const int r = a.prefix_mode ? static_cast<int>(blockIdx.z) / a.nsplit : static_cast<int>(blockIdx.z);
+  const int split = a.prefix_mode ? static_cast<int>(blockIdx.z) % a.nsplit : 0;
   const int qb = static_cast<int>(gridDim.x) - 1 - static_cast<int>(blockIdx.x);  // heaviest first
 
   // ---- block-uniform work description (identical in every thread) ---------
-  const int32_t p = a.prefix_lens[r], e = a.extend_lens[r];
+  const int32_t p = a.prefix_lens[r];
   const int64_t qbase = a.q_offsets[r];
+  const int32_t e = a.prefix_mode ? static_cast<int32_t>(a.q_offsets[r + 1] - qbase) : a.extend_lens[r];
   if (p < 0 || e < 0 || qbase < 0 || qbase + e > a.total_q) {
     if (threadIdx.x == 0 && blockIdx.x == 0 && g == 0) set_err(a.err, PKV_DEV_ERR_BAD_LENGTH);
     return;
@@ -282,15 +297,31 @@ __global__ void __launch_bounds__(kThreads, 1)
     set_err(a.err, PKV_DEV_ERR_BAD_LENGTH);
   const int i0 = qb * (kQTiles * TQ);
   if (i0 >= e) return;
-  const int32_t trow = a.table_idx[r];
+  // Prefix mode reads the keys through the row of the group's first member.
+  const int32_t trow = a.table_idx[a.prefix_mode ? qbase : r];
   const bool row_ok = trow >= 0 && trow < a.table_rows;
-  int64_t kv_end = static_cast<int64_t>(p) + min(e, i0 + kQTiles * TQ);
+  // Keys key0 .. kv_end - 1 are this CTA's (key0 is a multiple of the step).
+  const int64_t key0 = a.prefix_mode ? static_cast<int64_t>(split) * a.split_keys : 0;
+  int64_t kv_end = a.prefix_mode ? min(static_cast<int64_t>(p), key0 + a.split_keys)
+                                 : static_cast<int64_t>(p) + min(e, i0 + kQTiles * TQ);
   if (kv_end > a.table_cols) {
     if (threadIdx.x == 0) set_err(a.err, PKV_DEV_ERR_TABLE_RANGE);
     kv_end = a.table_cols;
   }
   if (!row_ok && threadIdx.x == 0) set_err(a.err, PKV_DEV_ERR_TABLE_RANGE);
-  const int nsteps = static_cast<int>((kv_end + kKeysPerStep - 1) / kKeysPerStep);
+  if (kv_end <= key0) {
+    // Prefix mode only (a causal block always has a key): an empty split
+    // leaves an empty partial, (max, sum) = (-inf, 0), which the merge skips.
+    if (warp < kWarpLoad0) {
+      const int m = (warp & 3) * 32 + lane;
+      const int tok = i0 + (warp >> 2) * TQ + m / G;
+      if (tok < e)
+        a.pre_ml[(static_cast<int64_t>(split) * a.nreq + qbase + tok) * a.hq + g * G + m % G] =
+            make_float2(-INFINITY, 0.f);
+    }
+    return;
+  }
+  const int nsteps = static_cast<int>((kv_end - key0 + kKeysPerStep - 1) / kKeysPerStep);
 
   // ---- setup: barriers and TMEM ------------------------------------------------
   if (threadIdx.x == 0) {
@@ -350,7 +381,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto lookup = [&](int jj, int32_t (&sl)[2]) {
 #pragma unroll
       for (int u = 0; u < 2; ++u) {
-        const int64_t key = static_cast<int64_t>(jj) * kKeysPerStep + u * 32 + lane;
+        const int64_t key = key0 + static_cast<int64_t>(jj) * kKeysPerStep + u * 32 + lane;
         int64_t sv = -1;
         if (jj < nsteps && key < kv_end && row_ok) sv = token_slot(rowp, key, a.page_size, a.num_slots, a.err);
         sl[u] = sv >= 0 ? static_cast<int32_t>(sv) : dummy;
@@ -503,7 +534,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int tq = m / G, hh = m % G;
     const int tok = i0 + i * TQ + tq;
     const bool valid = tok < e;
-    const int64_t lim = valid ? static_cast<int64_t>(p) + tok + 1 : 1;  // keys < lim visible
+    // Keys < lim are visible: causal in extend, the whole split in prefix mode.
+    const int64_t lim = a.prefix_mode ? kv_end : (valid ? static_cast<int64_t>(p) + tok + 1 : 1);
     const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
     const uint32_t o_addr = tmem + lane_base + kColO + 128 * i;
     float m_run = -INFINITY;
@@ -516,7 +548,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool w = mbar_wait(&bars[kBarSFull + 2 * i + hf], (j >> 1) & 1);
       if (__any_sync(0xffffffffu, !w || *abort_flag != 0)) { ok = false; break; }
       tc_fence_after();
-      const int64_t kb = static_cast<int64_t>(j) * kKeysPerStep;
+      const int64_t kb = key0 + static_cast<int64_t>(j) * kKeysPerStep;
       // Keys kb .. kb + vis - 1 of this step are visible to this row.
       const int64_t vis64 = lim - kb;
       const int32_t vis = vis64 <= 0 ? 0 : (vis64 >= kKeysPerStep ? kKeysPerStep : static_cast<int32_t>(vis64));
@@ -592,7 +624,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool w = mbar_wait(&bars[kBarOFinal], 0);
     w = __all_sync(0xffffffffu, w);
     tc_fence_after();
-    if (w && ok) {
+    if (w && ok && a.prefix_mode) {
+      const int64_t row = (static_cast<int64_t>(split) * a.nreq + qbase + tok) * a.hq + g * G + hh;
+      float* dst = a.pre_o + row * kHeadDim;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        float o[32];
+        tmem_ld32(o_addr + c * 32, o);
+        if (valid) {
+#pragma unroll
+          for (int u = 0; u < 32; u += 4)
+            *reinterpret_cast<float4*>(dst + c * 32 + u) = make_float4(o[u], o[u + 1], o[u + 2], o[u + 3]);
+        }
+      }
+      if (valid) a.pre_ml[row] = make_float2(m_run, l_run);
+    } else if (w && ok) {
       const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
       __nv_bfloat16* dst = a.out + ((qbase + tok) * a.hq + g * G + hh) * kHeadDim;
 #pragma unroll 1
@@ -653,13 +699,14 @@ bool make_q_map(CUtensorMap* map, const void* q, int32_t hq, int64_t total_q, in
 
 template <int G>
 cudaError_t launch_g(const CUtensorMap& qm, const ExtendTcArgs& a,
-                     int32_t batch, int32_t max_extend, cudaStream_t s) {
+                     int64_t grid_z, int32_t max_extend, cudaStream_t s) {
   constexpr int TQ = kRowsPerTile / G;
   const int nqb = (max_extend + kQTiles * TQ - 1) / (kQTiles * TQ);
   static int smem_state[kMaxDevicesHost] = {};
   cudaError_t e = ensure_smem_limit(extend_tc_kernel<G>, kSmemBytes, smem_state);
   if (e != cudaSuccess) return e;
-  dim3 grid(nqb, a.hkv, batch);
+  if (grid_z > 65535) return cudaErrorInvalidValue;
+  dim3 grid(nqb, a.hkv, static_cast<unsigned>(grid_z));
   extend_tc_kernel<G><<<grid, kThreads, kSmemBytes, s>>>(qm, a);
   return cudaGetLastError();
 }
@@ -695,11 +742,64 @@ cudaError_t launch_extend_tc(const PoolView& pool, const TableView& t, const voi
   a.hkv = pool.num_kv_heads;
   a.scale_log2 = scale * kLog2e;
   a.err = err;
+  a.prefix_mode = 0;
+  a.nsplit = 1;
+  a.split_keys = 0;
+  a.nreq = 0;
+  a.pre_ml = nullptr;
+  a.pre_o = nullptr;
   switch (G) {
     case 1: return launch_g<1>(qm, a, batch, max_extend, s);
     case 2: return launch_g<2>(qm, a, batch, max_extend, s);
     case 4: return launch_g<4>(qm, a, batch, max_extend, s);
     case 8: return launch_g<8>(qm, a, batch, max_extend, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_extend_prefix(const PoolView& pool, const TableView& t, const void* q,
+                                 int32_t num_q_heads, const int32_t* table_idx,
+                                 const int32_t* group_offsets, const int32_t* group_prefix,
+                                 int32_t num_groups, int32_t batch, int32_t nsplit, int32_t split_keys,
+                                 float scale, float2* pre_ml, float* pre_o, int32_t* err, cudaStream_t s) {
+  if (batch == 0 || num_groups == 0 || nsplit == 0) return cudaSuccess;
+  if (split_keys % kKeysPerStep != 0) return cudaErrorInvalidValue;
+  const int G = num_q_heads / pool.num_kv_heads;
+  CUtensorMap qm;
+  if (!make_q_map(&qm, q, num_q_heads, batch, G)) return cudaErrorInvalidValue;
+  ExtendTcArgs a;
+  a.kbase = pool.k;
+  a.vbase = pool.v;
+  a.slot_stride_bytes = pool.slot_stride_bytes;
+  a.table = t.entries;
+  a.table_rows = t.rows;
+  a.table_cols = t.cols;
+  a.table_stride = t.row_stride;
+  a.page_size = pool.page_size;
+  a.num_slots = pool.num_slots;
+  a.table_idx = table_idx;
+  a.prefix_lens = group_prefix;
+  a.extend_lens = nullptr;
+  a.q_offsets = group_offsets;
+  a.total_q = batch;
+  a.max_extend = batch;
+  a.out = nullptr;
+  a.hq = num_q_heads;
+  a.hkv = pool.num_kv_heads;
+  a.scale_log2 = scale * kLog2e;
+  a.err = err;
+  a.prefix_mode = 1;
+  a.nsplit = nsplit;
+  a.split_keys = split_keys;
+  a.nreq = batch;
+  a.pre_ml = pre_ml;
+  a.pre_o = pre_o;
+  const int64_t gz = static_cast<int64_t>(num_groups) * nsplit;
+  switch (G) {
+    case 1: return launch_g<1>(qm, a, gz, batch, s);
+    case 2: return launch_g<2>(qm, a, gz, batch, s);
+    case 4: return launch_g<4>(qm, a, gz, batch, s);
+    case 8: return launch_g<8>(qm, a, gz, batch, s);
   }
   return cudaErrorInvalidValue;
 }

@@ -65,10 +65,21 @@ cudaError_t launch_gather_kv(const PoolView& pool, const TableView& t, const int
 // Split-KV decode.
 size_t decode_workspace_bytes(int32_t batch, int32_t num_q_heads, int grid);
 int decode_grid_size();
+// Cascade decode: the suffix pass's column offsets and the shared-prefix
+// partials the combine kernel merges ([nsplit][batch][hq] (max, sum) pairs and
+// [nsplit][batch][hq][128] fp32 rows).
+struct CascadeView {
+  const int32_t* kv_start;
+  const float2* pre_ml;
+  const float* pre_o;
+  int32_t nsplit;
+};
+
 cudaError_t launch_decode(const PoolView& pool, const TableView& t, const void* q,
                           int32_t num_q_heads, const int32_t* table_idx, const int32_t* seq_lens,
                           int32_t batch, float scale, void* out, void* workspace, int grid,
-                          int32_t* err, cudaStream_t s);
+                          int32_t* err, cudaStream_t s,
+                          const struct CascadeView* cascade = nullptr);
 
 // Extend: tcgen05 path (bf16) and CUDA-core path (fp32 check build).
 cudaError_t launch_extend_tc(const PoolView& pool, const TableView& t, const void* q,
@@ -76,6 +87,26 @@ cudaError_t launch_extend_tc(const PoolView& pool, const TableView& t, const voi
                              const int32_t* prefix_lens, const int32_t* extend_lens,
                              const int32_t* q_offsets, int32_t batch, int64_t total_q, int32_t max_extend,
                              float scale, void* out, int32_t* err, cudaStream_t s);
+
+cudaError_t launch_extend_prefix(const PoolView& pool, const TableView& t, const void* q,
+                                 int32_t num_q_heads, const int32_t* table_idx,
+                                 const int32_t* group_offsets, const int32_t* group_prefix,
+                                 int32_t num_groups, int32_t batch, int32_t nsplit, int32_t split_keys,
+                                 float scale, float2* pre_ml, float* pre_o, int32_t* err, cudaStream_t s);
+
+cudaError_t launch_cascade_prep(const int32_t* group_offsets, const int32_t* group_prefix,
+                                int32_t num_groups, const int32_t* seq_lens, int32_t batch,
+                                int64_t prefix_capacity, int32_t* kv_start, int32_t* err,
+                                cudaStream_t s);
+
+size_t cascade_workspace_bytes(int32_t batch, int32_t num_q_heads, int64_t max_prefix_len);
+
+cudaError_t launch_decode_cascade(const PoolView& pool, const TableView& t, const void* q,
+                                  int32_t num_q_heads, const int32_t* table_idx,
+                                  const int32_t* seq_lens, int32_t batch,
+                                  const int32_t* group_offsets, const int32_t* group_prefix,
+                                  int32_t num_groups, int64_t max_prefix_len, float scale, void* out,
+                                  void* workspace, int32_t* err, cudaStream_t s);
 cudaError_t launch_extend_simt(const PoolView& pool, const TableView& t, const void* q,
                                int32_t num_q_heads, const int32_t* table_idx,
                                const int32_t* prefix_lens, const int32_t* extend_lens,

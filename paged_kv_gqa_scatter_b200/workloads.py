@@ -638,3 +638,75 @@ def rope_store_step(dtype: str = BF16, positions=None, num_q_heads: int = 16,
     out_loc = rng.choice(num_slots, size=n, replace=False).astype(np.int32)
     return RopeStoreWorkload(name, spec, num_q_heads, 0, kp, vp, qkv, positions,
                              rotary_table(max_position), qw, kw, 1e-6, out_loc)
+
+
+# ---------------------------------------------------------------------------
+# Decode batches whose requests share prefixes, in groups.
+# ---------------------------------------------------------------------------
+@dataclasses.dataclass
+class GroupedDecode:
+    """A decode step plus its grouping: requests group_offsets[g] ..
+    group_offsets[g+1] - 1 share their first group_prefix_lens[g] slots."""
+    decode: DecodeWorkload
+    group_offsets: np.ndarray      # int32 [groups + 1]
+    group_prefix_lens: np.ndarray  # int32 [groups]
+
+
+def grouped_decode(dtype: str = BF16, groups=((0, 3), (1, 1), (63, 2), (64, 5), (65, 1),
+                                              (1000, 70), (2500, 4)),
+                   min_suffix: int = 0, max_suffix: int = 300, num_q_heads: int = 16,
+                   num_kv_heads: int = 8, page_size: int = 1, seed: Optional[int] = None,
+                   name: str = "grouped-decode") -> GroupedDecode:
+    """Groups given as (prefix_len, members).  Each group's prefix occupies its
+    own slots (pages), shared by every member's table row; each member then has
+    a private suffix of U{min..max} tokens plus the token this step stores
+    (so a member's context is prefix + suffix + 1).  With page_size > 1 the
+    prefix lengths are rounded up to whole pages."""
+    rng = np.random.Generator(np.random.PCG64(seed_for(7) if seed is None else seed))
+    P = page_size
+    plens = [int(-(-p // P) * P) for p, _ in groups]
+    members = [int(m) for _, m in groups]
+    B = int(sum(members))
+    suffix = rng.integers(min_suffix, max_suffix, size=B, endpoint=True).astype(np.int64) + 1
+    pages_needed = sum(p // P for p in plens) + int(sum(-(-s // P) for s in suffix))
+    num_pages = pages_needed + 8
+    num_slots = num_pages * P
+    page_perm = rng.permutation(num_pages).astype(np.int64)
+    nxt = 0
+
+    def take(n_tokens):
+        nonlocal nxt
+        k = -(-n_tokens // P)
+        ph = page_perm[nxt:nxt + k]
+        nxt += k
+        return (ph[:, None] * P + np.arange(P)[None, :]).reshape(-1)[:n_tokens]
+
+    seq = np.zeros(B, dtype=np.int32)
+    cols = int(max(plens) + suffix.max())
+    cols = -(-cols // P) * P
+    table = _token_table(B + 1, cols)
+    table_idx = rng.permutation(B).astype(np.int32)
+    off = np.zeros(len(groups) + 1, dtype=np.int32)
+    r = 0
+    for gi, (p, m) in enumerate(zip(plens, members)):
+        shared = take(p) if p else np.zeros(0, dtype=np.int64)
+        for _ in range(m):
+            row = table_idx[r]
+            table[row, :p] = shared
+            own = take(int(suffix[r]))
+            table[row, p:p + own.shape[0]] = own
+            seq[r] = p + own.shape[0]
+            r += 1
+        off[gi + 1] = r
+    spec = PoolSpec(1, num_slots, num_kv_heads, HEAD_DIM, P, dtype)
+    kp = _new_plane_dict(spec, [0])
+    vp = _new_plane_dict(spec, [0])
+    _fill_slots(rng, kp[0], np.arange(num_slots), dtype)
+    _fill_slots(rng, vp[0], np.arange(num_slots), dtype)
+    q = draw_values(rng, (B, num_q_heads, HEAD_DIM), dtype)
+    k_new = draw_values(rng, (B, spec.row_elems), dtype)
+    v_new = draw_values(rng, (B, spec.row_elems), dtype)
+    out_loc = np.array([table[table_idx[i], seq[i] - 1] for i in range(B)], dtype=np.int32)
+    dec = DecodeWorkload(name, spec, num_q_heads, 0, kp, vp, table, table_idx, seq, q, k_new,
+                         v_new, out_loc, 1.0 / math.sqrt(HEAD_DIM))
+    return GroupedDecode(dec, off, np.asarray(plens, dtype=np.int32))
