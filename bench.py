@@ -243,7 +243,8 @@ def run_decode(args, world, rank, local):
         wl = W.decode_qwen3_8b(num_pages=num_pages)
         layers = list(range(wl.pool.num_layers))
     else:
-        wl = W.decode_qwen3_06b(num_layers=args.pool_layers, layer=min(13, args.pool_layers - 1))
+        nl = 28 if args.pool_layers is None else args.pool_layers
+        wl = W.decode_qwen3_06b(num_layers=nl, layer=min(13, nl - 1))
         layers = [wl.layer]
     lib = _lib.load()
 
@@ -672,16 +673,29 @@ def run_chunked_prefill(args, world, rank, local):
     }
 
 
+def radix_unique_bytes(dec) -> int:
+    """Bytes a decode step must read at least once: the shared prefix's K/V
+    once, every request's own tokens, its table entries, q and out."""
+    row = dec.pool.num_kv_heads * 128 * 2 * 2
+    own = int((dec.seq_lens.astype(np.int64) - 4096).sum())
+    return (4096 + own) * row + int(dec.seq_lens.astype(np.int64).sum()) * 4 + 2 * dec.q.size * 2
+
+
 def run_radix(args, world, rank, local):
     """Radix shared-prefix serving on a 32-layer pool: one step = the extend of
     all 256 suffixes on every layer (store_kv + extend_attn per layer), then
-    decode step 1 on every layer (store_kv + decode_attn per layer)."""
+    decode step 1 on every layer (store_kv + decode, per layer).  The decode
+    is the cascade call (the shared prefix attended once for the whole batch)
+    unless --radix-decode plain; the other form is timed beside the step on
+    two layers for comparison."""
     import torch
     from paged_kv_gqa_scatter_b200 import api
     from paged_kv_gqa_scatter_b200 import workloads as W
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    rs = W.radix_shared_prefix()
+    # --pool-layers below 32 shrinks the pool (and the layers stepped) for
+    # profiling; the per-layer work is unchanged.
+    rs = W.radix_shared_prefix(num_layers=32 if args.pool_layers is None else min(32, args.pool_layers))
     ext = rs.extend
     dec = rs.decode_step(1)
     L = ext.pool.num_layers
@@ -705,9 +719,20 @@ def run_radix(args, world, rank, local):
     d_loc = torch.from_numpy(dec.out_loc).to(dev)
     d_out = torch.empty_like(d_q)
     ws = api.decode_workspace(dec.batch, dec.num_q_heads, device=dev)
+    g_off = torch.tensor([0, dec.batch], dtype=torch.int32, device=dev)
+    g_pre = torch.tensor([4096], dtype=torch.int32, device=dev)
+    cws = api.decode_cascade_workspace(dec.batch, dec.num_q_heads, 4096, device=dev)
     err = torch.zeros(1, dtype=torch.int32, device=dev)
     s = torch.cuda.current_stream(dev)
     ext_ev, dec_ev = [], []
+    cascade = args.radix_decode == "cascade"
+
+    def decode(l, use_cascade):
+        if use_cascade:
+            api.decode_attn_cascade(pool, l, d_q, table, d_ti, d_sl, g_off, g_pre, 4096, d_out, cws,
+                                    scale=dec.scale, dev_err=err)
+        else:
+            api.decode_attn(pool, l, d_q, table, d_ti, d_sl, d_out, ws, scale=dec.scale, dev_err=err)
 
     def step(record):
         for l in range(L):
@@ -724,7 +749,7 @@ def run_radix(args, world, rank, local):
             a = torch.cuda.Event(enable_timing=True) if record else None
             b = torch.cuda.Event(enable_timing=True) if record else None
             if record: a.record(s)
-            api.decode_attn(pool, l, d_q, table, d_ti, d_sl, d_out, ws, scale=dec.scale, dev_err=err)
+            decode(l, cascade)
             if record:
                 b.record(s)
                 dec_ev.append((a, b))
@@ -746,6 +771,18 @@ def run_radix(args, world, rank, local):
     ms = max_over_ranks(start.elapsed_time(stop), world)
     ext_ms = sum(a.elapsed_time(b) for a, b in ext_ev)
     dec_ms = sum(a.elapsed_time(b) for a, b in dec_ev)
+    # The other decode form on layers 0 and L-1, outside the timed step.
+    other = []
+    for l in (0, L - 1):
+        for rep_i in range(4):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(s)
+            decode(l, not cascade)
+            b.record(s)
+            if rep_i > 0:
+                other.append((a, b))
+    torch.cuda.synchronize()
+    other_ms = sorted(a.elapsed_time(b) for a, b in other)[len(other) // 2]
     ext_flops = _flops_extend(ext) * L * args.steps
     logical = decode_bytes(dec) * L * args.steps
     _, bf16, _, src = measured_peaks()
@@ -760,16 +797,22 @@ def run_radix(args, world, rank, local):
         "config": {"workload": "radix-prefix", "layers": L, "batch": ext.batch, "prefix": 4096,
                    "suffix_tokens": ext.total_q, "num_q_heads": ext.num_q_heads,
                    "num_kv_heads": ext.pool.num_kv_heads,
-                   "step": "per layer store_kv + extend_attn, then per layer store_kv + decode_attn (decode step 1)",
+                   "step": ("per layer store_kv + extend_attn, then per layer store_kv + "
+                            + ("decode_attn_cascade" if cascade else "decode_attn") + " (decode step 1)"),
                    "parallelism": f"replicas x{world}"},
         "extend": {"tflops": round(tf, 2), "ms_per_layer": round(ext_ms / (L * args.steps), 4),
                    "roofline": {"bound": "tensor", "achieved": round(tf, 2), "peak": bf16,
                                 "peak_source": src, "unit": "TFLOP/s", "frac": round(tf / bf16, 4)}},
-        "decode": {"ms_per_layer": round(dec_ms / (L * args.steps), 4),
+        "decode": {"call": "decode_attn_cascade" if cascade else "decode_attn",
+                   "ms_per_layer": round(dec_ms / (L * args.steps), 4),
                    "tok_per_s_per_layer": round(dec.batch * L * args.steps / (dec_ms / 1e3), 1),
                    "logical_gbs": round(logical / (dec_ms / 1e3) / 1e9, 1),
-                   "note": "logical bytes count the shared 4096-token prefix once per request; most of it is served from L2"},
-        "gpu_launches": args.steps * L * 5,
+                   "unique_bytes_per_layer": radix_unique_bytes(dec),
+                   "prefix_flops_per_layer": 4 * 128 * dec.num_q_heads * dec.batch * 4096,
+                   "other_call": "decode_attn" if cascade else "decode_attn_cascade",
+                   "other_ms_per_layer": round(other_ms, 4),
+                   "note": "logical bytes count the shared 4096-token prefix once per request"},
+        "gpu_launches": args.steps * L * (2 + (5 if cascade else 3)),
         "device_error_word": int(err.item()),
         "clocks": clk,
     }
@@ -826,9 +869,11 @@ def main():
     ap.add_argument("--workload", default="decode-qwen3-0.6b",
                     choices=["decode-qwen3-0.6b", "decode-qwen3-8b", "chunked-prefill", "radix-prefix"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--pool-layers", type=int, default=28,
-                    help="layers of the decode-qwen3-0.6b pool (28 as stated; fewer only for profiling)")
+    ap.add_argument("--pool-layers", type=int, default=None,
+                    help="pool layers of decode-qwen3-0.6b (28) or radix-prefix (32); fewer only for profiling")
     ap.add_argument("--no-extend", action="store_true")
+    ap.add_argument("--radix-decode", choices=["cascade", "plain"], default="cascade",
+                    help="decode call of the radix-prefix workload's step")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
