@@ -457,3 +457,81 @@ def pin_fused_store(orc):
 
 ALL_PINS += [pin_bf16_rounding, pin_rms_norm_closed_form, pin_rope_closed_form,
              pin_rope_relative_position, pin_fused_store]
+
+
+# ---------------------------------------------------------------------------
+# FP8 (E4M3) pool pins.
+# ---------------------------------------------------------------------------
+# Hand-derived codes: value -> code (sign | exponent field << 3 | mantissa),
+# exponent bias 7, subnormal quantum 2^-9, largest finite 448 = 0x7E.
+E4M3_CASES = [
+    (1.0, 0x38), (-1.0, 0xB8), (448.0, 0x7E), (500.0, 0x7E), (-1000.0, 0xFE),
+    (464.0, 0x7E),                 # halfway 448 / 480: ties to even, 448
+    (240.0, 0x77),                 # 1.875 * 2^7
+    (2.0 ** -6, 0x08),             # smallest normal
+    (2.0 ** -9, 0x01),             # smallest subnormal
+    (2.0 ** -10, 0x00),            # halfway 0 / 2^-9: ties to even, 0
+    (3 * 2.0 ** -10, 0x02),        # halfway 2^-9 / 2^-8: ties to even, 2^-8
+    (1.4 * 2.0 ** -9, 0x01), (1.6 * 2.0 ** -9, 0x02),
+    (1.0625, 0x38),                # halfway 1 / 1.125: even mantissa 0
+    (1.1875, 0x3A),                # halfway 1.125 / 1.25: even mantissa 2
+    (1.9375, 0x40),                # rounds up into the next binade: 2.0
+    (0.0, 0x00), (-0.0, 0x80), (-3.5, 0xC6),
+]
+
+
+def pin_e4m3_codes(orc):
+    got = orc.e4m3_encode(np.array([v for v, _ in E4M3_CASES]))
+    want = [c for _, c in E4M3_CASES]
+    assert [int(x) for x in got] == want, [(v, hex(int(g))) for (v, _), g in zip(E4M3_CASES, got)]
+
+
+def pin_e4m3_decode_table(orc):
+    """All 256 codes: the value of each, built here from the format's fields,
+    and encode(decode(c)) == c for every finite code."""
+    codes = np.arange(256, dtype=np.uint8)
+    dec = orc.e4m3_decode(codes)
+    for c in range(256):
+        s, e, m = c >> 7, (c >> 3) & 15, c & 7
+        if e == 15 and m == 7:
+            assert math.isnan(dec[c])
+            continue
+        v = (m / 8.0) * 2.0 ** -6 if e == 0 else (1 + m / 8.0) * 2.0 ** (e - 7)
+        assert dec[c] == (-v if s else v), (c, dec[c], v)
+    finite = np.array([c for c in range(256) if (c & 0x7F) != 0x7F], dtype=np.uint8)
+    assert np.array_equal(orc.e4m3_encode(orc.e4m3_decode(finite)), finite)
+
+
+def pin_fp8_quantize_scale(orc):
+    """The stored code is that of x * (1/s) in float32: with s = 2, 2.125 ->
+    1.0625 -> 1.0 (tie to even), 3.0 -> 1.5, -896 -> -448 (saturated)."""
+    got = orc.quantize(np.array([2.125, 3.0, -896.0], dtype=np.float32), 2.0)
+    assert [int(x) for x in got] == [0x38, 0x3C, 0xFE]
+    bf = _bits(np.array([2.125, 3.0]))
+    assert [int(x) for x in orc.quantize(bf, 2.0)] == [0x38, 0x3C]
+
+
+def pin_fp8_one_token_returns_dequantised_v(orc):
+    """Store through the FP8 pool, then a one-token decode returns the token's
+    dequantised V: code(v / s) * s, here exactly v for values that are E4M3
+    numbers times s."""
+    rng = np.random.default_rng(53)
+    Hkv, Hq, S = 2, 4, 16
+    ks, vs = 0.75, 1.5
+    grid = np.array([(1 + m / 8.0) * 2.0 ** e for e in range(-3, 3) for m in range(8)])
+    v_vals = rng.choice(grid, size=(1, Hkv * D)) * rng.choice([-1.0, 1.0], size=(1, Hkv * D)) * vs
+    k_vals = rng.standard_normal((1, Hkv * D)).astype(np.float32)
+    kp = {0: np.zeros((S, Hkv, D), dtype=np.uint8)}
+    vp = {0: np.zeros((S, Hkv, D), dtype=np.uint8)}
+    orc.store_kv_fp8(kp, vp, 0, k_vals, v_vals.astype(np.float32), [5], Hkv, D, ks, vs)
+    assert np.count_nonzero(vp[0][np.arange(S) != 5]) == 0
+    table = np.array([[5]], dtype=np.int32)
+    q = _bits(rng.standard_normal((1, Hq, D)))
+    out = orc.decode_attn(q, orc.dequant_planes(kp, ks), orc.dequant_planes(vp, vs), 0, table,
+                          [0], [1], 1, 0.1)
+    for h in range(Hq):
+        assert np.array_equal(out[0, h], v_vals[0].reshape(Hkv, D)[h // 2])
+
+
+ALL_PINS += [pin_e4m3_codes, pin_e4m3_decode_table, pin_fp8_quantize_scale,
+             pin_fp8_one_token_returns_dequantised_v]

@@ -42,13 +42,14 @@ def test_cascade_grouped_matches_oracle(hq, hkv):
     tol_check(from_dev(out), exp, W.BF16, f"cascade hq={hq}")
 
 
-def test_cascade_paged():
-    gd = W.grouped_decode(page_size=16, seed=21)
+@pytest.mark.parametrize("page_size", [16, 64])
+def test_cascade_paged(page_size):
+    gd = W.grouped_decode(page_size=page_size, seed=21)
     dd = DeviceDecode(gd.decode)
     out = _run_cascade(dd, gd.group_offsets, gd.group_prefix_lens)
     assert int(dd.err.item()) == 0
     exp, _ = oracle_decode(gd.decode)
-    tol_check(from_dev(out), exp, W.BF16, "cascade page_size 16")
+    tol_check(from_dev(out), exp, W.BF16, f"cascade page_size {page_size}")
 
 
 def test_cascade_whole_context_shared():

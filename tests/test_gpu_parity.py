@@ -126,12 +126,14 @@ def test_decode_small(dtype):
 
 
 @pytest.mark.parametrize("dtype", DTYPES)
-def test_decode_paged_small(dtype):
-    wl = W.decode_paged_small(dtype=dtype)
+@pytest.mark.parametrize("page_size,num_slots", [(16, 4096), (64, 4096), (3, 4095)])
+def test_decode_paged_small(dtype, page_size, num_slots):
+    """page_size 16, the TRT-LLM-style 64, and a non-power-of-two size."""
+    wl = W.decode_paged_small(dtype=dtype, page_size=page_size, num_slots=num_slots)
     d = DeviceDecode(wl)
     d.run()
     exp, _ = oracle_decode(wl)
-    tol_check(from_dev(d.out), exp, dtype, "decode-paged")
+    tol_check(from_dev(d.out), exp, dtype, f"decode-paged P={page_size}")
     assert _err(d.err) == 0
 
 
@@ -238,9 +240,9 @@ def test_decode_qwen3_8b_sampled():
 # extend_attn.
 # ---------------------------------------------------------------------------
 @pytest.mark.parametrize("dtype", DTYPES)
-@pytest.mark.parametrize("page_size", [1, 4])
-def test_extend_small(dtype, page_size):
-    wl = W.extend_small(dtype=dtype, page_size=page_size)
+@pytest.mark.parametrize("page_size,num_slots", [(1, 1024), (4, 1024), (64, 1024), (3, 1023)])
+def test_extend_small(dtype, page_size, num_slots):
+    wl = W.extend_small(dtype=dtype, page_size=page_size, num_slots=num_slots)
     d = DeviceExtend(wl)
     d.run()
     exp, _ = oracle_extend(wl)

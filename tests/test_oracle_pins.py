@@ -45,32 +45,46 @@ ROPE_MUTATIONS = {
 }
 
 
+# The same for the FP8 pool oracle.
+FP8_MUTATIONS = {
+    "e4m3_bias_off": ("normal = np.ldexp(1.0 + m / 8.0, e - 7)", "normal = np.ldexp(1.0 + m / 8.0, e - 8)"),
+    "e4m3_truncates": ("r = np.rint(a / q) * q", "r = np.floor(a / q) * q"),
+    "e4m3_no_saturation": ("r = np.minimum(r, E4M3_MAX)", "r = r"),
+    "e4m3_subnormal_quantum": ("e = np.maximum(ex - 1, -6)", "e = np.maximum(ex - 1, -7)"),
+    "quantize_divides": ("t = (xf * inv).astype(np.float32)", "t = (xf / inv).astype(np.float32)"),
+    "dequant_forgets_scale": ("e4m3_decode(planes[l]) * float(np.float32(scale))", "e4m3_decode(planes[l])"),
+}
+
+
 def _mutant(name):
-    """The oracle package with one planted mistake (in either module)."""
+    """The oracle package with one planted mistake (in any one module)."""
     base = os.path.dirname(oracle.__file__)
-    pa = open(os.path.join(base, "paged_attention.py")).read()
-    rn = open(os.path.join(base, "rope_norm.py")).read()
-    if name in MUTATIONS:
-        old, new = MUTATIONS[name]
-        assert pa.count(old) == 1, f"mutation {name} does not match the oracle source once"
-        pa = pa.replace(old, new)
-    else:
-        old, new = ROPE_MUTATIONS[name]
-        assert rn.count(old) == 1, f"mutation {name} does not match the oracle source once"
-        rn = rn.replace(old, new)
+    src = {m: open(os.path.join(base, m + ".py")).read()
+           for m in ("paged_attention", "rope_norm", "fp8_pool")}
+    for mod, table in (("paged_attention", MUTATIONS), ("rope_norm", ROPE_MUTATIONS),
+                       ("fp8_pool", FP8_MUTATIONS)):
+        if name in table:
+            old, new = table[name]
+            assert src[mod].count(old) == 1, f"mutation {name} does not match the oracle source once"
+            src[mod] = src[mod].replace(old, new)
     m1 = types.ModuleType(f"oracle_pa_{name}")
-    exec(compile(pa, f"<mutant {name} paged_attention>", "exec"), m1.__dict__)
+    exec(compile(src["paged_attention"], f"<mutant {name} paged_attention>", "exec"), m1.__dict__)
     m2 = types.ModuleType(f"oracle_rn_{name}")
     m2.__dict__["to_f64"] = m1.to_f64
-    rn = rn.replace("from .paged_attention import to_f64\n", "")
+    rn = src["rope_norm"].replace("from .paged_attention import to_f64\n", "")
     exec(compile(rn, f"<mutant {name} rope_norm>", "exec"), m2.__dict__)
+    m3 = types.ModuleType(f"oracle_fp8_{name}")
+    exec(compile(src["fp8_pool"], f"<mutant {name} fp8_pool>", "exec"), m3.__dict__)
     mod = types.ModuleType(f"oracle_mutant_{name}")
     for k in oracle.__all__:
-        mod.__dict__[k] = getattr(m1, k) if hasattr(m1, k) else getattr(m2, k)
+        for m in (m1, m2, m3):
+            if hasattr(m, k):
+                mod.__dict__[k] = getattr(m, k)
+                break
     return mod
 
 
-@pytest.mark.parametrize("name", sorted(MUTATIONS) + sorted(ROPE_MUTATIONS))
+@pytest.mark.parametrize("name", sorted(MUTATIONS) + sorted(ROPE_MUTATIONS) + sorted(FP8_MUTATIONS))
 def test_planted_mistake_is_caught(name):
     mod = _mutant(name)
     failed = []
