@@ -190,18 +190,23 @@ def decode_bytes(wl) -> int:
     rows (all KV heads), its page-table entry (one per token at page_size 1, one
     per page otherwise), the queries and the outputs."""
     B, Hq = wl.batch, wl.num_q_heads
-    esz = 2 if wl.pool.dtype == "bf16" else 4
+    esz = ESIZE[wl.pool.dtype]
+    io = ESIZE[wl.pool.io_dtype]
     n = wl.seq_lens.astype(np.int64)
     row = wl.pool.num_kv_heads * 128 * esz
     P = wl.pool.page_size
     table = int(n.sum()) * 4 if P == 1 else int(((n + P - 1) // P).sum()) * 4
-    return int(n.sum()) * 2 * row + table + 2 * B * Hq * 128 * esz + 8 * B
+    return int(n.sum()) * 2 * row + table + 2 * B * Hq * 128 * io + 8 * B
+
+
+ESIZE = {"bf16": 2, "f32": 4, "fp8": 1}
 
 
 def store_bytes(wl) -> int:
-    esz = 2 if wl.pool.dtype == "bf16" else 4
-    row = wl.pool.num_kv_heads * 128 * esz
-    return wl.batch * (4 * row + 4)
+    """Read each new K and V row (row dtype), write it to the pool (pool dtype)."""
+    row_in = wl.pool.num_kv_heads * 128 * ESIZE[wl.pool.io_dtype]
+    row_out = wl.pool.num_kv_heads * 128 * ESIZE[wl.pool.dtype]
+    return wl.batch * (2 * (row_in + row_out) + 4)
 
 
 def cpu_decode_sample(wl, budget_s: float = 12.0):
@@ -245,6 +250,8 @@ def run_decode(args, world, rank, local):
     else:
         nl = 28 if args.pool_layers is None else args.pool_layers
         wl = W.decode_qwen3_06b(num_layers=nl, layer=min(13, nl - 1))
+        if args.kv_dtype == "fp8":
+            wl = W.with_fp8_pool(wl)
         layers = [wl.layer]
     lib = _lib.load()
 
@@ -253,8 +260,17 @@ def run_decode(args, world, rank, local):
         return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
 
     spec = wl.pool
+    fp8 = spec.dtype == "fp8"
+
+    def tpool(a):  # host plane contents -> device tensor of the pool's type
+        if fp8:
+            return torch.from_numpy(np.ascontiguousarray(a)).to(dev).view(torch.float8_e4m3fn)
+        return tdev(a)
+
     pool = api.KVPool.empty(spec.num_layers, spec.num_slots, spec.num_kv_heads, page_size=spec.page_size,
-                            device=dev, zero=not isinstance(wl.k_planes, W.TiledPlane))
+                            device=dev, zero=not isinstance(wl.k_planes, W.TiledPlane),
+                            dtype=torch.float8_e4m3fn if fp8 else torch.bfloat16,
+                            k_scale=spec.k_scale, v_scale=spec.v_scale)
     if isinstance(wl.k_planes, W.TiledPlane):
         for plane, dst in ((wl.k_planes, pool.k), (wl.v_planes, pool.v)):
             blk = tdev(plane.block)
@@ -265,8 +281,8 @@ def run_decode(args, world, rank, local):
                 flat[s:s + m].copy_(blk[:m])
     else:
         for l in layers:
-            pool.k[l].copy_(tdev(wl.k_planes[l]))
-            pool.v[l].copy_(tdev(wl.v_planes[l]))
+            pool.k[l].copy_(tpool(wl.k_planes[l]))
+            pool.v[l].copy_(tpool(wl.v_planes[l]))
     table = api.PageTable(torch.from_numpy(wl.page_table).to(dev))
     table_idx = torch.from_numpy(wl.table_idx).to(dev)
     seq_lens = torch.from_numpy(wl.seq_lens).to(dev)
@@ -398,9 +414,11 @@ def run_decode(args, world, rank, local):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "bf16",
-        "data": "synthetic (seeded PCG64 N(0,1) values rounded to bf16; K x0.5)" if wl.name.endswith("0.6b")
-                else "synthetic (seeded PCG64 N(0,1) block tiled over the pool)",
+        "dtype": "fp8-e4m3 pool, bf16 q/out" if fp8 else "bf16",
+        "data": ("synthetic (seeded random E4M3 codes in the pool, scales 0.05 / 0.09; bf16 q and new rows)"
+                 if fp8 else
+                 "synthetic (seeded PCG64 N(0,1) values rounded to bf16; K x0.5)" if wl.name.endswith("0.6b")
+                 else "synthetic (seeded PCG64 N(0,1) block tiled over the pool)"),
         "config": {
             "workload": wl.name,
             "batch": wl.batch,
@@ -436,11 +454,11 @@ def run_decode(args, world, rank, local):
     if args.workload == "decode-qwen3-8b":
         result["config"]["alias_factor"] = round(getattr(wl, "alias_factor", 0.0), 3)
 
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not fp8:
         gbs, sample, _ = cpu_decode_sample(wl)
         result["cpu_baseline"] = {"value": round(gbs, 4), "unit": "GB/s", "cores": blas_threads(),
                                   "kind": "oracle", "sample": sample}
-    if not args.no_extend and args.workload == "decode-qwen3-0.6b":
+    if not args.no_extend and args.workload == "decode-qwen3-0.6b" and not fp8:
         result["extend"] = run_extend_measure(dev, warmup=3, iters=max(5, args.steps))
         result["qk_norm_rope_store"] = run_rope_measure(dev, iters=max(5, args.steps))
     return result
@@ -503,6 +521,10 @@ def run_rope_measure(dev, iters=10, warmup=3):
         out[name] = {"us": round(us, 3), "bytes": nbytes, "GB/s": round(gbs, 1),
                      "frac": round(gbs / hbm, 4), "peak": hbm, "peak_source": src,
                      "device_error_word": int(err.item())}
+        if n == 16384:
+            out[name]["traffic"] = recorded_traffic("qk_norm_rope_store_kernel",
+                                                    source_hash("rope_store.cu", "common.cuh"),
+                                                    "rope prefill 16384")
     return out
 
 
@@ -872,6 +894,8 @@ def main():
     ap.add_argument("--pool-layers", type=int, default=None,
                     help="pool layers of decode-qwen3-0.6b (28) or radix-prefix (32); fewer only for profiling")
     ap.add_argument("--no-extend", action="store_true")
+    ap.add_argument("--kv-dtype", choices=["bf16", "fp8"], default="bf16",
+                    help="pool element type of decode-qwen3-0.6b (fp8: scaled E4M3 codes, bf16 q/out)")
     ap.add_argument("--radix-decode", choices=["cascade", "plain"], default="cascade",
                     help="decode call of the radix-prefix workload's step")
     args = ap.parse_args()

@@ -35,8 +35,10 @@
  *   int32, may be NULL).  No kernel traps, asserts or waits without bound:
  *   each internal wait gives up after about one second and sets
  *   PKV_DEV_ERR_TIMEOUT.
- * Element types: bf16 (the product path) and fp32 (a check build of the same
- *   kernels for tighter numerical comparison).  head_dim must be 128.
+ * Element types: bf16 (the product path), fp32 (a check build of the same
+ *   kernels for tighter numerical comparison) and a scaled FP8 E4M3 pool
+ *   (store, gather, fused store and decode; see pkv_pool).  head_dim must
+ *   be 128.
  */
 #ifndef PKV_H_
 #define PKV_H_
@@ -70,7 +72,7 @@ typedef enum {
   PKV_DEV_ERR_POSITION = 64      /* a RoPE position outside [0, max_position)           */
 } pkv_device_error;
 
-typedef enum { PKV_DTYPE_BF16 = 0, PKV_DTYPE_F32 = 1 } pkv_dtype;
+typedef enum { PKV_DTYPE_BF16 = 0, PKV_DTYPE_F32 = 1, PKV_DTYPE_FP8_E4M3 = 2 } pkv_dtype;
 
 /*
  * The KV pool [P5 §4.4.3; §1.4].
@@ -84,6 +86,15 @@ typedef enum { PKV_DTYPE_BF16 = 0, PKV_DTYPE_F32 = 1 } pkv_dtype;
  * num_kv_heads*head_dim).  Slot s of page p and offset o is s = p*page_size
  * + o.  `k` and `v` must be 16-byte aligned and slot_stride*element_size a
  * multiple of 16.  The caller owns the planes.
+ *
+ * FP8 pool (dtype PKV_DTYPE_FP8_E4M3; not on the pages, which keep K/V in
+ * the model dtype): each plane element is an OCP E4M3 code (1 byte) standing
+ * for code_value * k_scale (K plane) or * v_scale (V plane).  Calls that
+ * write the pool take bf16 rows and store the code of x * (1 / scale)
+ * (float32 product, round to nearest even, saturated to +-448); decode reads
+ * the codes and takes q and returns out in bf16.  Extend and cascade decode
+ * return PKV_ERR_UNSUPPORTED for FP8 pools.  The scales must be finite and
+ * > 0; they are ignored for the other dtypes.
  */
 typedef struct {
   void* k;
@@ -96,6 +107,8 @@ typedef struct {
   int32_t head_dim;
   int32_t page_size;
   int32_t dtype; /* pkv_dtype */
+  float k_scale;  /* FP8 pools: dequantisation scale of the K plane */
+  float v_scale;  /* FP8 pools: dequantisation scale of the V plane */
 } pkv_pool;
 
 /*
@@ -130,11 +143,12 @@ const char* pkv_version(void);
  *
  *   pool.k[layer][out_loc[i]][:] = k[i*k_row_stride .. + Hkv*head_dim)
  *   pool.v[layer][out_loc[i]][:] = v[i*v_row_stride .. + Hkv*head_dim)
- *   for 0 <= i < n_tokens, as a bit copy in the pool's element type.
+ *   for 0 <= i < n_tokens, as a bit copy in the pool's element type (for an
+ *   FP8 pool: the E4M3 codes of the bf16 rows, see pkv_pool).
  *
- * k, v: device, element type = pool.dtype, row strides in elements (k and v
- *   are typically column slices of a fused qkv output); both pointers and
- *   strides must keep rows 16-byte aligned.
+ * k, v: device, element type = pool.dtype (bf16 for an FP8 pool), row
+ *   strides in elements (k and v are typically column slices of a fused qkv
+ *   output); both pointers and strides must keep rows 16-byte aligned.
  * out_loc: device, int32 (out_loc_is_i64 = 0) or int64 (= 1), n_tokens entries.
  *   Slots must be distinct within one call (the pages give every new token
  *   its own slot); an out-of-range slot is skipped and sets
@@ -164,17 +178,18 @@ int pkv_store_kv(const pkv_pool* pool, int32_t layer, const void* k, int64_t k_r
  *   x_{i+64} c + x_i s) with c, s = cos_sin_cache[pos][i], [pos][64 + i].
  *   The pages do not spell the pairing out; rotate-half is the reading taken.
  *
- * qkv: device, pool dtype, rows of (Hq + 2 Hkv) * 128 elements, row stride
- *   in elements; 16-byte aligned rows.
+ * qkv: device, pool dtype (bf16 for an FP8 pool), rows of (Hq + 2 Hkv) * 128
+ *   elements, row stride in elements; 16-byte aligned rows.
  * positions: device int32 (positions_is_i64 = 0) or int64 (= 1) [n_tokens];
  *   a position outside [0, max_position) zeroes that token's q and k rows and
  *   sets PKV_DEV_ERR_POSITION.
  * cos_sin_cache: device float32 [max_position][128] (64 cos then 64 sin),
  *   16-byte aligned.
- * q_norm_weight, k_norm_weight: device [128] in the pool dtype, or NULL.
+ * q_norm_weight, k_norm_weight: device [128] in the qkv dtype, or NULL.
  * out_loc: as for pkv_store_kv (distinct slots; out of range is skipped and
- *   flagged).  q_out: device [n_tokens][num_q_heads][128], pool dtype.
- * All arithmetic is fp32; outputs round to the pool type (nearest even).
+ *   flagged).  q_out: device [n_tokens][num_q_heads][128], qkv dtype.
+ * All arithmetic is fp32; outputs round to their type (nearest even; an FP8
+ * pool stores the E4M3 codes of k * (1 / k_scale) and v * (1 / v_scale)).
  */
 int pkv_qk_norm_rope_store(const pkv_pool* pool, int32_t layer, const void* qkv,
                            int64_t qkv_row_stride, int32_t num_q_heads, const void* positions,
@@ -213,8 +228,9 @@ int pkv_gather_kv(const pkv_pool* pool, int32_t layer, const pkv_page_table* tab
  *   over j < seq_lens[r], G = num_q_heads / pool.num_kv_heads,
  *   K_r[j] = pool.k[layer][slot(r, j)], V_r likewise.
  *
- * q: device [batch][num_q_heads][head_dim] contiguous, pool dtype.
- * out: device [batch][num_q_heads][head_dim] contiguous, pool dtype
+ * q: device [batch][num_q_heads][head_dim] contiguous, pool dtype (bf16 for
+ *   an FP8 pool, whose K/V are read as code * scale).
+ * out: device [batch][num_q_heads][head_dim] contiguous, q's dtype
  *   (fp32 accumulation, rounded to nearest-even on store).
  * table_idx, seq_lens: device int32 [batch].
  * scale: softmax scale (the pages do not state it; 1/sqrt(head_dim) is the

@@ -23,7 +23,8 @@ c_size = ctypes.c_size_t
 class PkvPool(ctypes.Structure):
     _fields_ = [("k", c_vp), ("v", c_vp), ("num_layers", c_i64), ("num_slots", c_i64),
                 ("layer_stride", c_i64), ("slot_stride", c_i64), ("num_kv_heads", c_i32),
-                ("head_dim", c_i32), ("page_size", c_i32), ("dtype", c_i32)]
+                ("head_dim", c_i32), ("page_size", c_i32), ("dtype", c_i32),
+                ("k_scale", ctypes.c_float), ("v_scale", ctypes.c_float)]
 
 
 class PkvPageTable(ctypes.Structure):

@@ -15,7 +15,7 @@ import torch
 
 from . import _lib
 
-DTYPE_CODES = {torch.bfloat16: 0, torch.float32: 1}
+DTYPE_CODES = {torch.bfloat16: 0, torch.float32: 1, torch.float8_e4m3fn: 2}
 HEAD_DIM = 128
 
 # pkv_device_error bits OR-ed into a call's dev_err word.
@@ -50,7 +50,8 @@ class KVPool:
     slot's heads and dims are contiguous (the pool layout of include/pkv.h).
     """
 
-    def __init__(self, k: torch.Tensor, v: torch.Tensor, page_size: int = 1):
+    def __init__(self, k: torch.Tensor, v: torch.Tensor, page_size: int = 1,
+                 k_scale: float = 1.0, v_scale: float = 1.0):
         if k.shape != v.shape or k.dtype != v.dtype or k.dim() != 4:
             raise ValueError("k and v must be matching 4-D tensors")
         if k.stride(3) != 1 or k.stride(2) != k.shape[3] or v.stride() != k.stride():
@@ -63,15 +64,22 @@ class KVPool:
         self.c = _lib.PkvPool(
             k=k.data_ptr(), v=v.data_ptr(), num_layers=k.shape[0], num_slots=k.shape[1],
             layer_stride=k.stride(0), slot_stride=k.stride(1), num_kv_heads=k.shape[2],
-            head_dim=k.shape[3], page_size=self.page_size, dtype=DTYPE_CODES[k.dtype])
+            head_dim=k.shape[3], page_size=self.page_size, dtype=DTYPE_CODES[k.dtype],
+            k_scale=float(k_scale), v_scale=float(v_scale))
+        self.k_scale, self.v_scale = float(k_scale), float(v_scale)
 
     @classmethod
     def empty(cls, num_layers, num_slots, num_kv_heads, dtype=torch.bfloat16, page_size=1,
-              device="cuda", zero=True):
+              device="cuda", zero=True, k_scale=1.0, v_scale=1.0):
         mk = torch.zeros if zero else torch.empty
         k = mk((num_layers, num_slots, num_kv_heads, HEAD_DIM), dtype=dtype, device=device)
         v = mk((num_layers, num_slots, num_kv_heads, HEAD_DIM), dtype=dtype, device=device)
-        return cls(k, v, page_size)
+        return cls(k, v, page_size, k_scale, v_scale)
+
+    @property
+    def io_dtype(self):
+        """dtype of the rows a call writes into the pool, and of q / out."""
+        return torch.bfloat16 if self.k.dtype == torch.float8_e4m3fn else self.k.dtype
 
     @property
     def num_kv_heads(self) -> int:
@@ -102,8 +110,8 @@ def store_kv(pool: KVPool, layer: int, k: torch.Tensor, v: torch.Tensor, out_loc
         k = k.reshape(k.shape[0], -1)
     if v.dim() == 3:
         v = v.reshape(v.shape[0], -1)
-    if k.stride(1) != 1 or v.stride(1) != 1 or k.dtype != pool.dtype or v.dtype != pool.dtype:
-        raise ValueError("k/v rows must be contiguous and of the pool dtype")
+    if k.stride(1) != 1 or v.stride(1) != 1 or k.dtype != pool.io_dtype or v.dtype != pool.io_dtype:
+        raise ValueError("k/v rows must be contiguous and of the pool's row dtype")
     if out_loc.dtype not in (torch.int32, torch.int64) or not out_loc.is_contiguous():
         raise ValueError("out_loc must be contiguous int32 or int64")
     lib = _lib.load()
@@ -120,8 +128,8 @@ def qk_norm_rope_store(pool: KVPool, layer: int, qkv: torch.Tensor, num_q_heads:
                        dev_err: Optional[torch.Tensor] = None, stream=None) -> None:
     """pkv_qk_norm_rope_store: q/k RMSNorm + RoPE, then k/v into the pool, q into q_out."""
     _require_cuda(qkv, positions, cos_sin_cache, out_loc, q_out, q_norm_weight, k_norm_weight, dev_err)
-    if qkv.dim() != 2 or qkv.dtype != pool.dtype or (qkv.shape[0] > 0 and qkv.stride(1) != 1):
-        raise ValueError("qkv must be [tokens][(Hq + 2 Hkv) * 128] rows of the pool dtype")
+    if qkv.dim() != 2 or qkv.dtype != pool.io_dtype or (qkv.shape[0] > 0 and qkv.stride(1) != 1):
+        raise ValueError("qkv must be [tokens][(Hq + 2 Hkv) * 128] rows of the pool's row dtype")
     if cos_sin_cache.dtype != torch.float32 or not cos_sin_cache.is_contiguous():
         raise ValueError("cos_sin_cache must be contiguous float32 [max_position][128]")
     for t, name in ((positions, "positions"), (out_loc, "out_loc")):
@@ -165,7 +173,7 @@ def decode_attn(pool: KVPool, layer: int, q: torch.Tensor, table: PageTable,
     _require_cuda(q, table_idx, seq_lens, out, workspace, dev_err)
     if not (q.is_contiguous() and out.is_contiguous()):
         raise ValueError("q and out must be contiguous")
-    if q.dtype != pool.dtype or out.dtype != pool.dtype:
+    if q.dtype != pool.io_dtype or out.dtype != pool.io_dtype:
         raise ValueError("q/out dtype must match the pool")
     B, Hq, D = q.shape
     scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
@@ -189,7 +197,7 @@ def decode_attn_noalloc(pool: KVPool, layer: int, q: torch.Tensor, table: PageTa
     _require_cuda(q, table_idx, seq_lens, out, dev_err)
     if not (q.is_contiguous() and out.is_contiguous()):
         raise ValueError("q and out must be contiguous")
-    if q.dtype != pool.dtype or out.dtype != pool.dtype:
+    if q.dtype != pool.io_dtype or out.dtype != pool.io_dtype:
         raise ValueError("q/out dtype must match the pool")
     B, Hq, D = q.shape
     scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
@@ -221,7 +229,7 @@ def decode_attn_cascade(pool: KVPool, layer: int, q: torch.Tensor, table: PageTa
     _require_cuda(q, table_idx, seq_lens, group_offsets, group_prefix_lens, out, workspace, dev_err)
     if not (q.is_contiguous() and out.is_contiguous()):
         raise ValueError("q and out must be contiguous")
-    if q.dtype != pool.dtype or out.dtype != pool.dtype:
+    if q.dtype != pool.io_dtype or out.dtype != pool.io_dtype:
         raise ValueError("q/out dtype must match the pool")
     for t, name in ((group_offsets, "group_offsets"), (group_prefix_lens, "group_prefix_lens")):
         if t.dtype != torch.int32 or not t.is_contiguous():
@@ -250,7 +258,7 @@ def extend_attn(pool: KVPool, layer: int, q: torch.Tensor, table: PageTable,
     _require_cuda(q, table_idx, prefix_lens, extend_lens, q_offsets, out, workspace, dev_err)
     if not (q.is_contiguous() and out.is_contiguous()):
         raise ValueError("q and out must be contiguous")
-    if q.dtype != pool.dtype or out.dtype != pool.dtype:
+    if q.dtype != pool.io_dtype or out.dtype != pool.io_dtype:
         raise ValueError("q/out dtype must match the pool")
     T, Hq, D = q.shape
     scale = 1.0 / math.sqrt(D) if scale is None else float(scale)

@@ -23,8 +23,15 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 int esize_of(int32_t dtype) {
   if (dtype == PKV_DTYPE_BF16) return 2;
   if (dtype == PKV_DTYPE_F32) return 4;
+  if (dtype == PKV_DTYPE_FP8_E4M3) return 1;
   return 0;
 }
+
+// Element size of the rows a call reads or writes beside the pool (k/v to
+// store, qkv, q, out): bf16 for an FP8 pool, the pool's type otherwise.
+int io_esize(const PoolView& pv) { return pv.dtype == PKV_DTYPE_FP8_E4M3 ? 2 : pv.esize; }
+
+bool finite_positive(float x) { return x > 0.f && x <= 3.402823466e38f; }
 
 int check_pool(const pkv_pool* p, int32_t layer, PoolView* out) {
   if (p == nullptr || p->k == nullptr || p->v == nullptr) return PKV_ERR_INVALID_ARG;
@@ -34,6 +41,8 @@ int check_pool(const pkv_pool* p, int32_t layer, PoolView* out) {
   if (p->num_kv_heads < 1 || p->num_layers < 1 || p->num_slots < 1 || p->page_size < 1)
     return PKV_ERR_INVALID_ARG;
   if (layer < 0 || layer >= p->num_layers) return PKV_ERR_INVALID_ARG;
+  if (p->dtype == PKV_DTYPE_FP8_E4M3 && !(finite_positive(p->k_scale) && finite_positive(p->v_scale)))
+    return PKV_ERR_INVALID_ARG;
   const int64_t row = static_cast<int64_t>(p->num_kv_heads) * p->head_dim;
   if (p->slot_stride < row || p->layer_stride < 0) return PKV_ERR_INVALID_ARG;
   if (p->num_layers > 1 && p->layer_stride < p->num_slots * p->slot_stride) return PKV_ERR_INVALID_ARG;
@@ -51,6 +60,8 @@ int check_pool(const pkv_pool* p, int32_t layer, PoolView* out) {
   out->page_size = p->page_size;
   out->esize = es;
   out->dtype = p->dtype;
+  out->k_scale = p->dtype == PKV_DTYPE_FP8_E4M3 ? p->k_scale : 1.f;
+  out->v_scale = p->dtype == PKV_DTYPE_FP8_E4M3 ? p->v_scale : 1.f;
   return PKV_OK;
 }
 
@@ -107,10 +118,11 @@ int pkv_store_kv(const pkv_pool* pool, int32_t layer, const void* k, int64_t k_r
   const int64_t row = static_cast<int64_t>(pool->num_kv_heads) * pool->head_dim;
   if (k_row_stride < row || v_row_stride < row) return PKV_ERR_INVALID_ARG;
   if (out_loc_is_i64 != 0 && out_loc_is_i64 != 1) return PKV_ERR_INVALID_ARG;
-  if (!aligned16(k) || !aligned16(v) || (k_row_stride * pv.esize) % 16 != 0 ||
-      (v_row_stride * pv.esize) % 16 != 0)
+  const int ies = io_esize(pv);
+  if (!aligned16(k) || !aligned16(v) || (k_row_stride * ies) % 16 != 0 ||
+      (v_row_stride * ies) % 16 != 0)
     return PKV_ERR_MISALIGNED;
-  return from_cuda(pkv::launch_store_kv(pv, k, k_row_stride * pv.esize, v, v_row_stride * pv.esize,
+  return from_cuda(pkv::launch_store_kv(pv, k, k_row_stride * ies, v, v_row_stride * ies,
                                         out_loc, out_loc_is_i64 == 1, n_tokens, dev_err,
                                         static_cast<cudaStream_t>(stream)));
 }
@@ -134,7 +146,7 @@ int pkv_qk_norm_rope_store(const pkv_pool* pool, int32_t layer, const void* qkv,
   if (!(eps >= 0.f)) return PKV_ERR_INVALID_ARG;
   const int64_t row = static_cast<int64_t>(num_q_heads + 2 * pool->num_kv_heads) * pool->head_dim;
   if (qkv_row_stride < row) return PKV_ERR_INVALID_ARG;
-  if (!aligned16(qkv) || (qkv_row_stride * pv.esize) % 16 != 0 || !aligned16(q_out) ||
+  if (!aligned16(qkv) || (qkv_row_stride * io_esize(pv)) % 16 != 0 || !aligned16(q_out) ||
       !aligned16(cos_sin_cache) || (q_norm_weight && !aligned16(q_norm_weight)) ||
       (k_norm_weight && !aligned16(k_norm_weight)))
     return PKV_ERR_MISALIGNED;
@@ -262,6 +274,7 @@ int pkv_extend_attn(const pkv_pool* pool, int32_t layer, const void* q, int32_t 
   if (!q || !out || !table_idx || !prefix_lens || !extend_lens || !q_offsets)
     return PKV_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(out)) return PKV_ERR_MISALIGNED;
+  if (pv.dtype == PKV_DTYPE_FP8_E4M3) return PKV_ERR_UNSUPPORTED;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (pv.dtype == PKV_DTYPE_BF16)
     return from_cuda(pkv::launch_extend_tc(pv, tv, q, num_q_heads, table_idx, prefix_lens,

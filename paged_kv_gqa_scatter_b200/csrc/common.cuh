@@ -6,6 +6,8 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -55,6 +57,34 @@ __device__ __forceinline__ void load8<float>(const float* p, float2 (&f)[4]) {
   f[1] = make_float2(a.z, a.w);
   f[2] = make_float2(b.x, b.y);
   f[3] = make_float2(b.z, b.w);
+}
+
+template <>
+__device__ __forceinline__ void load8<__nv_fp8_e4m3>(const __nv_fp8_e4m3* p, float2 (&f)[4]) {
+  // E4M3 codes widen exactly to half, then to float.
+  const uint2 w = *reinterpret_cast<const uint2*>(p);
+  const uint32_t u[2] = {w.x, w.y};
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const __half2_raw lo = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(u[i] & 0xffffu), __NV_E4M3);
+    const __half2_raw hi = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(u[i] >> 16), __NV_E4M3);
+    f[2 * i] = __half22float2(*reinterpret_cast<const __half2*>(&lo));
+    f[2 * i + 1] = __half22float2(*reinterpret_cast<const __half2*>(&hi));
+  }
+}
+
+// Two floats -> two E4M3 codes (round to nearest even, saturated to +-448),
+// a in the low byte.
+__device__ __forceinline__ uint32_t pack_e4m3x2(float a, float b) {
+  return static_cast<uint32_t>(__nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3));
+}
+
+// 8 floats times inv_scale (float32 products) -> 8 E4M3 codes.
+__device__ __forceinline__ uint2 quant8_e4m3(const float (&f)[8], float inv_scale) {
+  uint2 w;
+  w.x = pack_e4m3x2(f[0] * inv_scale, f[1] * inv_scale) | (pack_e4m3x2(f[2] * inv_scale, f[3] * inv_scale) << 16);
+  w.y = pack_e4m3x2(f[4] * inv_scale, f[5] * inv_scale) | (pack_e4m3x2(f[6] * inv_scale, f[7] * inv_scale) << 16);
+  return w;
 }
 
 // Store 8 floats as 8 elements (bf16: round to nearest even).

@@ -43,15 +43,24 @@ constexpr int kStages = 3;
 constexpr int kMinTokensPerCta = 32;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
+// Per pool element type: tokens per ring stage (a stage holds 2 x T rows of
+// Hkv x 128 elements, 64 KB at Hkv 8) and the type of q and out.
 template <typename E>
 struct DecodeTraits;
 template <>
 struct DecodeTraits<__nv_bfloat16> {
   static constexpr int kTokensPerStage = 16;
+  using IO = __nv_bfloat16;
 };
 template <>
 struct DecodeTraits<float> {
   static constexpr int kTokensPerStage = 8;
+  using IO = float;
+};
+template <>
+struct DecodeTraits<__nv_fp8_e4m3> {  // E4M3 codes; q and out stay bf16
+  static constexpr int kTokensPerStage = 32;
+  using IO = __nv_bfloat16;
 };
 
 struct DecodeArgs {
@@ -68,7 +77,8 @@ struct DecodeArgs {
   const void* q;
   void* out;
   int32_t hq, hkv;
-  float scale_log2;
+  float scale_log2;   // softmax scale * log2(e) * K dequantisation scale
+  float v_scale;      // V dequantisation scale (FP8 pools; 1 otherwise)
   int32_t row_bytes;  // Hkv * 128 * esize
   int32_t* ws_cum;    // [batch + 1]
   int64_t* ws_per;    // [1]
@@ -138,6 +148,7 @@ __global__ void __launch_bounds__(32 * 9, 1) decode_split_kernel(const DecodeArg
   constexpr int NV = V >= 16 ? V / 16 : 1;         // complete sums per lane after reduce
   constexpr int LPH = 16 / G;                      // lanes per head within a half
   constexpr int ESZ = sizeof(E);
+  using IO = typename DecodeTraits<E>::IO;
   constexpr int kLog2V = V >= 16 ? 4 : (V == 8 ? 3 : (V == 4 ? 2 : (V == 2 ? 1 : 0)));
 
   extern __shared__ __align__(128) uint8_t smem[];
@@ -357,8 +368,8 @@ __global__ void __launch_bounds__(32 * 9, 1) decode_split_kernel(const DecodeArg
   if (g >= ncons) return;
   const int c = lane & 15, half = lane >> 4;
   float* pw = psm + g * SUB * G;  // this warp's p buffer [SUB][G]
-  const E* qbase = static_cast<const E*>(a.q);
-  E* obase = static_cast<E*>(a.out);
+  const IO* qbase = static_cast<const IO*>(a.q);
+  IO* obase = static_cast<IO*>(a.out);
   int64_t s = 0;
   for (int r = rfirst; r < B && cum[r] < hi; ++r) {
     const int64_t ja = max(lo, (int64_t)cum[r]) - cum[r];
@@ -368,12 +379,12 @@ __global__ void __launch_bounds__(32 * 9, 1) decode_split_kernel(const DecodeArg
     // Warm L2 with the next request's queries while this piece runs.
     if (r + 1 < B && cum[r + 1] < hi && lane < 2 * G)
       asm volatile("prefetch.global.L2 [%0];" ::"l"(qbase + ((int64_t)(r + 1) * a.hq + g * G) * kHeadDim +
-                                                      lane * (128 / ESZ)));
+                                                      lane * (128 / static_cast<int>(sizeof(IO)))));
 
     float2 q2[G][4];
 #pragma unroll
     for (int hh = 0; hh < G; ++hh) {
-      load8<E>(qbase + ((int64_t)r * a.hq + g * G + hh) * kHeadDim + 8 * c, q2[hh]);
+      load8<IO>(qbase + ((int64_t)r * a.hq + g * G + hh) * kHeadDim + 8 * c, q2[hh]);
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         q2[hh][e].x *= a.scale_log2;
@@ -498,6 +509,15 @@ __global__ void __launch_bounds__(32 * 9, 1) decode_split_kernel(const DecodeArg
         o2[hh][e].y += __shfl_xor_sync(0xffffffffu, o2[hh][e].y, 16);
       }
     }
+    if constexpr (sizeof(E) == 1) {  // FP8 pool: V codes stand for code * v_scale
+#pragma unroll
+      for (int hh = 0; hh < G; ++hh)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          o2[hh][e].x *= a.v_scale;
+          o2[hh][e].y *= a.v_scale;
+        }
+    }
     float mh[G];
 #pragma unroll
     for (int hh = 0; hh < G; ++hh) mh[hh] = __shfl_sync(0xffffffffu, m_run, hh * LPH);
@@ -513,7 +533,7 @@ __global__ void __launch_bounds__(32 * 9, 1) decode_split_kernel(const DecodeArg
           f[2 * e] = o2[hh][e].x * inv;
           f[2 * e + 1] = o2[hh][e].y * inv;
         }
-        store8<E>(obase + ((int64_t)r * a.hq + h) * kHeadDim + 8 * c, f);
+        store8<IO>(obase + ((int64_t)r * a.hq + h) * kHeadDim + 8 * c, f);
       } else {
         const int64_t id = static_cast<int64_t>(blockIdx.x) + r;
         float* op = a.ws_o + (id * a.hq + h) * kHeadDim + 8 * c;
@@ -627,7 +647,8 @@ cudaError_t launch_decode_t(const DecodeArgs& a, int grid, cudaStream_t s, const
   ccfg.gridDim = dim3(a.batch, (a.hq + 3) / 4);
   ccfg.blockDim = dim3(128);
   ccfg.dynamicSmemBytes = 0;
-  return cudaLaunchKernelEx(&ccfg, decode_combine_kernel<E>, a.seq_lens, (const int32_t*)a.ws_cum,
+  return cudaLaunchKernelEx(&ccfg, decode_combine_kernel<typename DecodeTraits<E>::IO>, a.seq_lens,
+                            (const int32_t*)a.ws_cum,
                             (const int64_t*)a.ws_per, (const float2*)a.ws_ml, (const float*)a.ws_o,
                             a.hq, a.out, cv ? cv->pre_ml : nullptr, cv ? cv->pre_o : nullptr,
                             cv ? cv->nsplit : 0);
@@ -675,7 +696,8 @@ cudaError_t launch_decode(const PoolView& pool, const TableView& t, const void* 
   a.out = out;
   a.hq = num_q_heads;
   a.hkv = pool.num_kv_heads;
-  a.scale_log2 = scale * kLog2e;
+  a.scale_log2 = scale * kLog2e * pool.k_scale;
+  a.v_scale = pool.v_scale;
   a.row_bytes = pool.num_kv_heads * kHeadDim * pool.esize;
   uint8_t* w = static_cast<uint8_t*>(workspace);
   a.ws_per = reinterpret_cast<int64_t*>(w);
@@ -691,7 +713,14 @@ cudaError_t launch_decode(const PoolView& pool, const TableView& t, const void* 
   a.kv_start = cascade ? cascade->kv_start : nullptr;
   a.cascade = cascade ? 1 : 0;
   const int G = num_q_heads / pool.num_kv_heads;
-  if (pool.dtype == PKV_DTYPE_BF16) {
+  if (pool.dtype == PKV_DTYPE_FP8_E4M3) {
+    switch (G) {
+      case 1: return launch_decode_t<__nv_fp8_e4m3, 1>(a, grid, s, cascade);
+      case 2: return launch_decode_t<__nv_fp8_e4m3, 2>(a, grid, s, cascade);
+      case 4: return launch_decode_t<__nv_fp8_e4m3, 4>(a, grid, s, cascade);
+      case 8: return launch_decode_t<__nv_fp8_e4m3, 8>(a, grid, s, cascade);
+    }
+  } else if (pool.dtype == PKV_DTYPE_BF16) {
     switch (G) {
       case 1: return launch_decode_t<__nv_bfloat16, 1>(a, grid, s, cascade);
       case 2: return launch_decode_t<__nv_bfloat16, 2>(a, grid, s, cascade);

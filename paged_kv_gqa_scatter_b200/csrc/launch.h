@@ -39,6 +39,7 @@ struct PoolView {
   int32_t page_size;
   int32_t esize;  // element size in bytes
   int32_t dtype;
+  float k_scale, v_scale;  // FP8 dequantisation scales (1 otherwise)
 };
 
 struct TableView {

@@ -43,6 +43,7 @@ struct RopeArgs {
   int64_t n;
   void* q_out;              // [n][hq][128]
   int32_t* err;
+  float k_inv, v_inv;       // FP8 pool: 1 / dequantisation scale
 };
 
 // 8 elements as raw 16-byte words (one for bf16, two for fp32), so that a v
@@ -96,8 +97,11 @@ __device__ __forceinline__ void load_w8(const void* w, int c, float (&f)[8]) {
 // rows with that stride, kRif rows at a time: every row load of a group is
 // issued before any of them is used, and the token's position, slot and
 // cos/sin values are loaded once per half-warp, not once per row.
-template <typename E, int kThreads, int kRif, int kMinBlocks>
+// kFp8: the pool holds E4M3 codes; k and v rows are stored as the codes of
+// value * (1 / scale) (E is then bf16, the type of qkv and q_out).
+template <typename E, int kThreads, int kRif, int kMinBlocks, bool kFp8>
 __global__ void __launch_bounds__(kThreads, kMinBlocks) qk_norm_rope_store_kernel(const RopeArgs a) {
+  constexpr int kPoolEsize = kFp8 ? 1 : static_cast<int>(sizeof(E));
   constexpr int kHalfWarps = kThreads / 16;
   const int64_t t = blockIdx.x;
   const int rows = a.hq + 2 * a.hkv;
@@ -145,11 +149,17 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) qk_norm_rope_store_kerne
       const int r = r0 + kHalfWarps * u;
       if (r >= rows) break;
       const int kind = r < a.hq ? 0 : (r < a.hq + a.hkv ? 1 : 2);  // q, k, v
-      if (kind == 2) {  // v: bit copy into the pool
+      if (kind == 2) {  // v: bit copy into the pool (FP8: its codes)
         if (slot_ok) {
-          E* dst = reinterpret_cast<E*>(a.vpool + slot * a.slot_stride_bytes) +
-                   (r - a.hq - a.hkv) * kHeadDim + 8 * c;
-          store_raw8<E>(dst, raw[u]);
+          uint8_t* dst = a.vpool + slot * a.slot_stride_bytes +
+                         ((r - a.hq - a.hkv) * kHeadDim + 8 * c) * kPoolEsize;
+          if constexpr (kFp8) {
+            float xv[8];
+            to_floats(raw[u], xv);
+            *reinterpret_cast<uint2*>(dst) = quant8_e4m3(xv, a.v_inv);
+          } else {
+            store_raw8<E>(reinterpret_cast<E*>(dst), raw[u]);
+          }
         }
         continue;
       }
@@ -177,8 +187,11 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) qk_norm_rope_store_kerne
       if (kind == 0) {
         store8<E>(static_cast<E*>(a.q_out) + (t * a.hq + r) * kHeadDim + 8 * c, y);
       } else if (slot_ok) {
-        store8<E>(reinterpret_cast<E*>(a.kpool + slot * a.slot_stride_bytes) +
-                      (r - a.hq) * kHeadDim + 8 * c, y);
+        uint8_t* dst = a.kpool + slot * a.slot_stride_bytes + ((r - a.hq) * kHeadDim + 8 * c) * kPoolEsize;
+        if constexpr (kFp8)
+          *reinterpret_cast<uint2*>(dst) = quant8_e4m3(y, a.k_inv);
+        else
+          store8<E>(reinterpret_cast<E*>(dst), y);
       }
     }
   }
@@ -218,10 +231,14 @@ cudaError_t launch_qk_norm_rope_store(const PoolView& pool, const void* qkv, int
   // 64-thread blocks (4 half-warps, 4 rows in flight each) at 16 blocks per
   // SM: measured best on B200 among 32-512 threads and 2-8 rows in flight
   // (about 96% of copy bandwidth at 32k tokens of Hq 32 / Hkv 8).
+  a.k_inv = 1.0f / pool.k_scale;
+  a.v_inv = 1.0f / pool.v_scale;
   if (pool.dtype == PKV_DTYPE_BF16)
-    qk_norm_rope_store_kernel<__nv_bfloat16, 64, 4, 16><<<blocks, 64, 0, s>>>(a);
+    qk_norm_rope_store_kernel<__nv_bfloat16, 64, 4, 16, false><<<blocks, 64, 0, s>>>(a);
+  else if (pool.dtype == PKV_DTYPE_FP8_E4M3)
+    qk_norm_rope_store_kernel<__nv_bfloat16, 64, 4, 16, true><<<blocks, 64, 0, s>>>(a);
   else
-    qk_norm_rope_store_kernel<float, 64, 2, 16><<<blocks, 64, 0, s>>>(a);
+    qk_norm_rope_store_kernel<float, 64, 2, 16, false><<<blocks, 64, 0, s>>>(a);
   return cudaGetLastError();
 }
 

@@ -34,6 +34,7 @@ import numpy as np
 HEAD_DIM = 128
 BF16 = "bf16"
 F32 = "f32"
+F8 = "fp8"  # scaled E4M3 pool: uint8 codes on the host; q / k / v rows stay bf16
 
 
 def seed_for(workload_number: int) -> int:
@@ -66,7 +67,17 @@ def draw_values(rng: np.random.Generator, shape, dtype: str, scale: float = 1.0)
 
 
 def storage_dtype(dtype: str):
-    return np.uint16 if dtype == BF16 else np.float32
+    return {BF16: np.uint16, F32: np.float32, F8: np.uint8}[dtype]
+
+
+def draw_e4m3_codes(rng: np.random.Generator, shape, min_exp: int = 4, max_exp: int = 9) -> np.ndarray:
+    """Random E4M3 codes: sign and mantissa uniform, exponent field uniform in
+    [min_exp, max_exp] (values of magnitude 2^(min_exp-7) .. < 2^(max_exp-6));
+    never a NaN code.  Drawn directly as codes, so no rounding is involved."""
+    sign = rng.integers(0, 2, size=shape, dtype=np.uint8) << np.uint8(7)
+    ex = rng.integers(min_exp, max_exp, size=shape, dtype=np.uint8, endpoint=True) << np.uint8(3)
+    man = rng.integers(0, 8, size=shape, dtype=np.uint8)
+    return sign | ex | man
 
 
 class TiledPlane:
@@ -131,6 +142,13 @@ class PoolSpec:
     head_dim: int
     page_size: int
     dtype: str
+    k_scale: float = 1.0  # F8 pools: dequantisation scales
+    v_scale: float = 1.0
+
+    @property
+    def io_dtype(self) -> str:
+        """Element type of q, out and the rows written into the pool."""
+        return BF16 if self.dtype == F8 else self.dtype
 
     @property
     def row_elems(self) -> int:
@@ -710,3 +728,23 @@ def grouped_decode(dtype: str = BF16, groups=((0, 3), (1, 1), (63, 2), (64, 5), 
     dec = DecodeWorkload(name, spec, num_q_heads, 0, kp, vp, table, table_idx, seq, q, k_new,
                          v_new, out_loc, 1.0 / math.sqrt(HEAD_DIM))
     return GroupedDecode(dec, off, np.asarray(plens, dtype=np.int32))
+
+
+# ---------------------------------------------------------------------------
+# FP8 (scaled E4M3) pools.
+# ---------------------------------------------------------------------------
+def with_fp8_pool(wl: DecodeWorkload, k_scale: float = 0.05, v_scale: float = 0.09,
+                  seed: Optional[int] = None) -> DecodeWorkload:
+    """The same decode step over an E4M3 pool: every slot of the touched layers
+    holds random codes (see draw_e4m3_codes); q and the new K/V rows stay the
+    bf16 values of ``wl``; the scales are not powers of two, so the stored
+    codes of the new rows depend on float32 rounding of x * (1 / scale)."""
+    rng = np.random.Generator(np.random.PCG64(seed_for(8) if seed is None else seed))
+    if wl.pool.dtype != BF16 or isinstance(wl.k_planes, TiledPlane):
+        raise ValueError("needs a bf16 workload with dict planes")
+    spec = dataclasses.replace(wl.pool, dtype=F8, k_scale=float(np.float32(k_scale)),
+                               v_scale=float(np.float32(v_scale)))
+    shape = (spec.num_slots, spec.num_kv_heads, spec.head_dim)
+    kp = {l: draw_e4m3_codes(rng, shape) for l in wl.k_planes}
+    vp = {l: draw_e4m3_codes(rng, shape) for l in wl.v_planes}
+    return dataclasses.replace(wl, name=wl.name + "-fp8", pool=spec, k_planes=kp, v_planes=vp)

@@ -15,13 +15,15 @@ import oracle
 from paged_kv_gqa_scatter_b200 import api
 from paged_kv_gqa_scatter_b200 import workloads as W
 
-TORCH_DTYPE = {W.BF16: torch.bfloat16, W.F32: torch.float32}
+TORCH_DTYPE = {W.BF16: torch.bfloat16, W.F32: torch.float32, W.F8: torch.float8_e4m3fn}
 
 
 def to_dev(arr: np.ndarray, dtype: str, device="cuda") -> torch.Tensor:
-    """Host element array (bf16 bits or float32) -> device tensor of the element type."""
+    """Host element array (bf16 bits, float32, or E4M3 codes) -> device tensor of the element type."""
     if dtype == W.BF16:
         return torch.from_numpy(np.ascontiguousarray(arr).view(np.int16)).view(torch.bfloat16).to(device)
+    if dtype == W.F8:
+        return torch.from_numpy(np.ascontiguousarray(arr, dtype=np.uint8)).to(device).view(torch.float8_e4m3fn)
     return torch.from_numpy(np.ascontiguousarray(arr, dtype=np.float32)).to(device)
 
 
@@ -39,7 +41,8 @@ def device_pool(spec: W.PoolSpec, k_planes, v_planes, layers=None) -> api.KVPool
     ``layers`` (default: every layer the host planes hold)."""
     dt = TORCH_DTYPE[spec.dtype]
     pool = api.KVPool.empty(spec.num_layers, spec.num_slots, spec.num_kv_heads, dtype=dt,
-                            page_size=spec.page_size, zero=True)
+                            page_size=spec.page_size, zero=True, k_scale=spec.k_scale,
+                            v_scale=spec.v_scale)
     if isinstance(k_planes, W.TiledPlane):
         lay = range(spec.num_layers) if layers is None else layers
         for plane, dst in ((k_planes, pool.k), (v_planes, pool.v)):
@@ -90,7 +93,7 @@ class DeviceDecode:
 
     def __init__(self, wl: W.DecodeWorkload, pool: api.KVPool = None, table=None):
         self.wl = wl
-        dt = wl.pool.dtype
+        dt = wl.pool.io_dtype
         self.pool = pool if pool is not None else device_pool(wl.pool, wl.k_planes, wl.v_planes,
                                                               layers=[wl.layer])
         self.table = table if table is not None else api.PageTable(i32(wl.page_table))

@@ -1,0 +1,174 @@
+"""GPU parity for the scaled FP8 (E4M3) KV pool against the oracle.
+
+* store_kv / gather: the stored codes are bit-exact (both sides quantise the
+  float32 product x * RN32(1 / scale) with round-to-nearest-even).
+* decode: attention over the dequantised pool, |err| <= 1e-2 + 1e-2 |ref|.
+* fused norm/RoPE/store: v codes bit-exact (a bf16 value times the inverse
+  scale is the same float32 product on both sides); k codes come from an
+  fp32 kernel value and a float64 oracle value, so they may differ by one
+  code where the two straddle a rounding boundary: the dequantised k must be
+  within one E4M3 step (2^-3 relative, or 2^-9 * scale near zero) and 97% of
+  the codes must agree.
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gpu_helpers import DeviceDecode, device_pool, from_dev, i32, to_dev, tol_check
+from paged_kv_gqa_scatter_b200 import api
+from paged_kv_gqa_scatter_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+D = W.HEAD_DIM
+
+
+def _codes(t: torch.Tensor) -> np.ndarray:
+    return t.view(torch.uint8).cpu().numpy()
+
+
+def _oracle_store(wl):
+    kp = {l: a.copy() for l, a in wl.k_planes.items()}
+    vp = {l: a.copy() for l, a in wl.v_planes.items()}
+    oracle.store_kv_fp8(kp, vp, wl.layer, wl.k_new, wl.v_new, wl.out_loc, wl.pool.num_kv_heads, D,
+                        wl.pool.k_scale, wl.pool.v_scale)
+    return kp, vp
+
+
+def _oracle_decode(wl, kp, vp, requests=None):
+    return oracle.decode_attn(wl.q, oracle.dequant_planes(kp, wl.pool.k_scale, [wl.layer]),
+                              oracle.dequant_planes(vp, wl.pool.v_scale, [wl.layer]), wl.layer,
+                              wl.page_table, wl.table_idx, wl.seq_lens, wl.pool.page_size, wl.scale,
+                              requests=requests)
+
+
+@pytest.mark.parametrize("loc64", [False, True])
+def test_fp8_store_codes_bit_exact(loc64):
+    wl = W.with_fp8_pool(W.decode_small())
+    d = DeviceDecode(wl)
+    loc = d.out_loc.long() if loc64 else d.out_loc
+    api.store_kv(d.pool, 0, d.k_new, d.v_new, loc, d.err)
+    torch.cuda.synchronize()
+    assert int(d.err.item()) == 0
+    kp, vp = _oracle_store(wl)
+    assert np.array_equal(_codes(d.pool.k[0]), kp[0])
+    assert np.array_equal(_codes(d.pool.v[0]), vp[0])
+
+
+def test_fp8_store_saturates():
+    """Rows far beyond 448 * scale store the largest code, with its sign."""
+    wl = W.with_fp8_pool(W.decode_small(), k_scale=0.001, v_scale=0.001)
+    d = DeviceDecode(wl)
+    api.store_kv(d.pool, 0, d.k_new, d.v_new, d.out_loc, d.err)
+    torch.cuda.synchronize()
+    kp, vp = _oracle_store(wl)
+    got = _codes(d.pool.k[0])
+    assert np.array_equal(got, kp[0])
+    rows = got[wl.out_loc]
+    assert np.any((rows & 0x7F) == 0x7E)  # some values did saturate
+
+
+def test_fp8_gather_bit_exact():
+    wl = W.with_fp8_pool(W.decode_paged_small(), seed=3)
+    d = DeviceDecode(wl)
+    B = wl.batch
+    offs = np.zeros(B + 1, dtype=np.int64)
+    offs[1:] = np.cumsum(wl.seq_lens)
+    total = int(offs[-1])
+    ko = torch.empty((total, wl.pool.num_kv_heads, D), dtype=torch.float8_e4m3fn, device="cuda")
+    vo = torch.empty_like(ko)
+    api.gather_kv(d.pool, 0, d.table, d.table_idx, d.seq_lens, torch.from_numpy(offs).cuda(), ko, vo, d.err)
+    torch.cuda.synchronize()
+    rows = oracle.gather_kv(wl.k_planes, wl.v_planes, 0, wl.page_table, wl.table_idx, wl.seq_lens,
+                            wl.pool.page_size)
+    assert np.array_equal(_codes(ko), np.concatenate([kr for kr, _ in rows]))
+    assert np.array_equal(_codes(vo), np.concatenate([vr for _, vr in rows]))
+
+
+@pytest.mark.parametrize("maker,hq", [("decode_small", 16), ("decode_small", 32), ("decode_small", 8),
+                                      ("decode_small", 64), ("decode_paged_small", 32)])
+def test_fp8_decode_matches_oracle(maker, hq):
+    base = getattr(W, maker)(num_q_heads=hq) if maker == "decode_small" else W.decode_paged_small()
+    wl = W.with_fp8_pool(base, seed=hq)
+    d = DeviceDecode(wl)
+    d.run()
+    torch.cuda.synchronize()
+    assert int(d.err.item()) == 0
+    kp, vp = _oracle_store(wl)
+    exp = _oracle_decode(wl, kp, vp)
+    tol_check(from_dev(d.out), exp, W.BF16, f"fp8 decode {maker} hq={hq}")
+
+
+def test_fp8_decode_qwen3_06b_full():
+    """The bench's decode step over an E4M3 copy of its pool (64 requests,
+    141,622 context tokens, Hq 16, Hkv 8)."""
+    wl = W.with_fp8_pool(W.decode_qwen3_06b(num_layers=1, layer=0))
+    d = DeviceDecode(wl)
+    d.run()
+    torch.cuda.synchronize()
+    assert int(d.err.item()) == 0
+    kp, vp = _oracle_store(wl)
+    rng = np.random.default_rng(9)
+    req = sorted(rng.choice(wl.batch, 12, replace=False).tolist())
+    exp = _oracle_decode(wl, kp, vp, requests=req)
+    tol_check(from_dev(d.out)[req], exp[req], W.BF16, "fp8 decode-qwen3-0.6b")
+
+
+def test_fp8_rope_store():
+    wl = W.rope_store_step(W.BF16, seed=31)
+    hq, hkv = wl.num_q_heads, wl.pool.num_kv_heads
+    ks, vs = float(np.float32(0.02)), float(np.float32(0.03))
+    spec = W.PoolSpec(1, wl.pool.num_slots, hkv, D, 1, W.F8, ks, vs)
+    rng = np.random.Generator(np.random.PCG64(77))
+    kp0 = {0: W.draw_e4m3_codes(rng, (spec.num_slots, hkv, D))}
+    vp0 = {0: W.draw_e4m3_codes(rng, (spec.num_slots, hkv, D))}
+    pool = device_pool(spec, kp0, vp0)
+    qkv = to_dev(wl.qkv, W.BF16)
+    q_out = torch.empty((wl.n_tokens, hq, D), dtype=torch.bfloat16, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    api.qk_norm_rope_store(pool, 0, qkv, hq, i32(wl.positions), torch.from_numpy(wl.cos_sin_cache).cuda(),
+                           i32(wl.out_loc), q_out, to_dev(wl.q_norm_w, W.BF16), to_dev(wl.k_norm_w, W.BF16),
+                           wl.eps, err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    # Oracle: q and k in float64 (bf16 planes as scratch), v codes by quantize.
+    kb = {0: np.zeros((spec.num_slots, hkv, D), dtype=np.uint16)}
+    vb = {0: np.zeros((spec.num_slots, hkv, D), dtype=np.uint16)}
+    q = oracle.qk_norm_rope_store(wl.qkv, hq, hkv, D, wl.positions, wl.cos_sin_cache, wl.q_norm_w,
+                                  wl.k_norm_w, wl.eps, kb, vb, 0, wl.out_loc, storage="bf16")
+    x = oracle.to_f64(wl.qkv).reshape(wl.n_tokens, hq + 2 * hkv, D)
+    k = oracle.rope_rotate_half(oracle.rms_norm(x[:, hq:hq + hkv], wl.k_norm_w, wl.eps), wl.positions,
+                                wl.cos_sin_cache)
+    v_codes = oracle.quantize(wl.qkv[:, (hq + hkv) * D:], vs).reshape(wl.n_tokens, hkv, D)
+    # q_out as in the bf16 path.
+    got_q = from_dev(q_out)
+    assert np.all(np.abs(got_q - q) <= 2.0 ** -8 * np.abs(q) + 2.0 ** -18 * np.abs(q).max(axis=-1, keepdims=True))
+    gk = _codes(pool.k[0])[wl.out_loc]
+    gv = _codes(pool.v[0])[wl.out_loc]
+    assert np.array_equal(gv, v_codes)
+    kdeq = oracle.e4m3_decode(gk) * ks
+    bound = 2.0 ** -3 * np.abs(k) + 2.0 ** -9 * ks
+    assert np.all(np.abs(kdeq - k) <= bound)
+    same = np.mean(gk == oracle.quantize(k.astype(np.float32), ks).reshape(gk.shape))
+    assert same >= 0.97, same
+    # Every other slot is untouched.
+    others = np.setdiff1d(np.arange(spec.num_slots), wl.out_loc)
+    assert np.array_equal(_codes(pool.k[0])[others], kp0[0][others])
+    assert np.array_equal(_codes(pool.v[0])[others], vp0[0][others])
+
+
+def test_fp8_unsupported_calls():
+    wl = W.with_fp8_pool(W.decode_small())
+    d = DeviceDecode(wl)
+    out = torch.empty_like(d.q)
+    qo = torch.tensor([0, 1], dtype=torch.int32, device="cuda")
+    with pytest.raises(RuntimeError, match="unsupported"):
+        api.extend_attn(d.pool, 0, d.q[:1], d.table, d.table_idx[:1], i32([0]), i32([1]), qo, 1,
+                        out[:1], scale=wl.scale)
+    ws = api.decode_cascade_workspace(wl.batch, wl.num_q_heads, 16)
+    with pytest.raises(RuntimeError, match="unsupported"):
+        api.decode_attn_cascade(d.pool, 0, d.q, d.table, d.table_idx, d.seq_lens, i32([0, wl.batch]),
+                                i32([16]), 16, out, ws, scale=wl.scale)
