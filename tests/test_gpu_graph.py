@@ -96,3 +96,99 @@ def test_decode_graph_ladder_with_dummy_padding():
             torch.cuda.synchronize()
             tol_check(from_dev(out[:B]), expected[idx], W.BF16, f"graph bs={bs} real={B}")
     assert int(err.item()) == 0
+
+
+def _capture(fn):
+    """Warm up eagerly once, then capture fn in a CUDA graph."""
+    fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    with torch.cuda.graph(g, stream=s):
+        fn()
+    torch.cuda.synchronize()
+    return g
+
+
+def test_fused_store_then_cascade_decode_in_graph():
+    """qk_norm_rope_store followed by decode_attn_cascade, captured once and
+    replayed with two different qkv inputs in the same fixed buffer: each
+    replay equals (bit for bit) the same two calls run eagerly, and the
+    eager result matches the oracle's store and decode."""
+    import oracle
+    gd = W.grouped_decode(groups=((128, 6), (700, 10)), max_suffix=200, seed=61)
+    d = gd.decode
+    Hq, Hkv, B = d.num_q_heads, d.pool.num_kv_heads, d.batch
+    rng = np.random.Generator(np.random.PCG64(62))
+    pos_np = (d.seq_lens - 1).astype(np.int32)
+    cache_np = W.rotary_table(4096)
+    qw_np = W.f32_to_bf16_bits(1.0 + 0.1 * rng.standard_normal(128).astype(np.float32))
+    kw_np = W.f32_to_bf16_bits(1.0 + 0.1 * rng.standard_normal(128).astype(np.float32))
+    qkv_a = W.draw_values(rng, (B, (Hq + 2 * Hkv) * 128), W.BF16, 2.0)
+    qkv_b = W.draw_values(rng, (B, (Hq + 2 * Hkv) * 128), W.BF16, 2.0)
+    mp = int(gd.group_prefix_lens.max())
+    table = api.PageTable(i32(d.page_table))
+    ti, sl, loc, pos = i32(d.table_idx), i32(d.seq_lens), i32(d.out_loc), i32(pos_np)
+    off, pre = i32(gd.group_offsets), i32(gd.group_prefix_lens)
+    cache = torch.from_numpy(cache_np).cuda()
+    qw, kw = to_dev(qw_np, W.BF16), to_dev(kw_np, W.BF16)
+
+    def make():
+        pool = device_pool(d.pool, d.k_planes, d.v_planes, layers=[0])
+        qkv = torch.empty((B, (Hq + 2 * Hkv) * 128), dtype=torch.bfloat16, device="cuda")
+        q_out = torch.empty((B, Hq, 128), dtype=torch.bfloat16, device="cuda")
+        out = torch.empty((B, Hq, 128), dtype=torch.bfloat16, device="cuda")
+        ws = api.decode_cascade_workspace(B, Hq, mp)
+        err = torch.zeros(1, dtype=torch.int32, device="cuda")
+
+        def fn():
+            api.qk_norm_rope_store(pool, 0, qkv, Hq, pos, cache, loc, q_out, qw, kw, 1e-6, err)
+            api.decode_attn_cascade(pool, 0, q_out, table, ti, sl, off, pre, mp, out, ws,
+                                    scale=d.scale, dev_err=err)
+        return qkv, out, err, fn
+
+    qkv_e, out_e, err_e, fn_e = make()
+    qkv_g, out_g, err_g, fn_g = make()
+    qkv_g.copy_(to_dev(qkv_a, W.BF16))
+    g = _capture(fn_g)
+    for host in (qkv_a, qkv_b):
+        qkv_e.copy_(to_dev(host, W.BF16))
+        fn_e()
+        qkv_g.copy_(to_dev(host, W.BF16))
+        out_g.fill_(0)
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(out_e, out_g)
+    assert int(err_e.item()) == 0 and int(err_g.item()) == 0
+    # The eager result of the second input against the oracle.
+    kp = {0: d.k_planes[0].copy()}
+    vp = {0: d.v_planes[0].copy()}
+    q = oracle.qk_norm_rope_store(qkv_b, Hq, Hkv, 128, pos_np, cache_np, qw_np, kw_np, 1e-6, kp, vp, 0,
+                                  d.out_loc)
+    exp = oracle.decode_attn(oracle.to_storage(q, "bf16"), kp, vp, 0, d.page_table, d.table_idx,
+                             d.seq_lens, 1, d.scale)
+    tol_check(from_dev(out_e), exp, W.BF16, "fused store + cascade decode")
+
+
+def test_fp8_store_and_decode_in_graph():
+    """store_kv + decode_attn over an FP8 pool, captured and replayed twice;
+    each replay equals the eager calls bit for bit."""
+    wl = W.with_fp8_pool(W.decode_small(num_q_heads=32), seed=63)
+
+    def make():
+        from gpu_helpers import DeviceDecode
+        dd = DeviceDecode(wl)
+        return dd, dd.run
+
+    de, fe = make()
+    dg, fg = make()
+    g = _capture(fg)
+    for scale in (1.0, -0.5):
+        for dd in (de, dg):
+            dd.q.copy_(to_dev(wl.q, W.BF16) * scale)
+        fe()
+        dg.out.fill_(0)
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(de.out, dg.out)
+    assert int(de.err.item()) == 0 and int(dg.err.item()) == 0
