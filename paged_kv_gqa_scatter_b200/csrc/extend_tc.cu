@@ -13,29 +13,34 @@
 //  * A CTA owns one (request, KV head, 2 x 128 query rows) block.  Rows are
 //    (token, query head of the group) pairs, token-major, so the G query heads
 //    sharing a KV head form the M dimension of one MMA and every K/V tile is
-//    used by 256 rows.
-//  * warps 8 and 9 -- K/V loads: each warp owns one stage of a 2-deep ring
-//    and loads every other tile.  For each 128-key tile a warp translates the keys'
-//    slots through the page table (one tile ahead) and moves the 256-byte head
-//    rows with 16-byte cp.async copies straight into the 128-byte-swizzled
-//    UMMA operand layout: K-major for K (B of Q K^T), MN-major for V (B of
-//    P V).  A lane pair of half-warps covers two rows per step, so every warp
-//    access is two fully used 256-byte segments.  (TMA tile::gather4 was tried
-//    first: four 128-byte rows per instruction issued too slowly to feed the
-//    tensor core.)
+//    used by 256 rows.  The grid is (KV head, query block, request) with the
+//    heaviest query block first, and blocks are dispatched in that linear
+//    order, so the longest CTAs start first.
+//  * warps 8 and 9 -- K/V loads in 64-key steps through a 4-stage ring; warp
+//    8 loads the even steps, warp 9 the odd ones.  For each step a warp
+//    translates the keys' slots through the page table (one step ahead) and
+//    moves the 256-byte head rows with 16-byte cp.async copies straight into
+//    the 128-byte-swizzled UMMA operand layout: K-major for K (B of Q K^T),
+//    MN-major for V (B of P V).  Two half-warps cover two rows per
+//    instruction, so every warp access is two fully used 256-byte segments.
+//    (TMA tile::gather4 was tried first: four 128-byte rows per instruction
+//    issued too slowly to feed the tensor core.)
 //  * warp 10 -- the two Q tiles by 3-D TMA boxes [tokens][G heads][64 dims]
-//    (128-byte swizzle), TMEM allocation, and MMA issue (one thread):
-//    S_i = Q_i K^T into TMEM (M=128, N=128, K=16 steps), then O_i += P_i V with
-//    P_i read from TMEM.  Issue order PV_0(j), QK_0(j+1), PV_1(j), QK_1(j+1)
-//    lets softmax of one Q tile run while the tensor core works on the other.
+//    (128-byte swizzle), TMEM allocation, and MMA issue: S_i = Q_i K^T into
+//    TMEM (M=128, N=64, K=16 steps), then O_i += P_i V (N=128) with P_i read
+//    from TMEM.  The whole warp runs the issue loop so descriptors stay
+//    warp-uniform; one elected lane issues.  Issue order PV_0(j), QK_0(j+2),
+//    PV_1(j), QK_1(j+2): scores are always two steps ahead of the softmax.
 //    Completion is signalled with tcgen05.commit to mbarriers.
-//  * warps 0-3 and 4-7 -- softmax for Q tile 0 and 1: one thread per row,
-//    the S row read from TMEM in one go, log2-domain online softmax with a lazily moved
-//    max (O rescaled in TMEM only when the max grows by more than 2^8), P
-//    written back over S as packed bf16 with tcgen05.st; at the end O / l is
-//    read from TMEM and stored as bf16.
-//  * TMEM (512 columns): S_0, S_1, O_0, O_1, 128 fp32 columns each; P_i
-//    occupies the first 64 columns of S_i.
+//  * warps 0-3 and 4-7 -- softmax for Q tile 0 and 1: one thread per row, the
+//    step's 64 scores read from TMEM in one go, log2-domain online softmax
+//    with a lazily moved max (O rescaled in TMEM only when the max grows by
+//    more than 2^8), P written back over S as packed bf16 with tcgen05.st; at
+//    the end O / l is read from TMEM and stored as bf16 (prefix mode: O and
+//    (max, sum) as fp32 partials).
+//  * TMEM (512 columns): S_0 and S_1 as two 64-column halves each (double
+//    buffered by step parity), O_0, O_1 128 fp32 columns each; P overwrites
+//    the first 32 columns of its S half.
 //  * Every mbarrier wait is bounded (about one second); on a timeout the CTA
 //    records PKV_DEV_ERR_TIMEOUT, drains its copies and MMAs, frees TMEM and
 //    returns.
@@ -280,20 +285,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int32_t* abort_flag = reinterpret_cast<volatile int32_t*>(smem + kOffMisc + 16);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int g = blockIdx.y;
+  const int g = blockIdx.x;
   const int r = a.prefix_mode ? static_cast<int>(blockIdx.z) / a.nsplit : static_cast<int>(blockIdx.z);
   const int split = a.prefix_mode ? static_cast<int>(blockIdx.z) % a.nsplit : 0;
-  const int qb = static_cast<int>(gridDim.x) - 1 - static_cast<int>(blockIdx.x);  // heaviest first
+  // Blocks are dispatched in linear order (x fastest): all KV heads of the
+  // heaviest query block first, so the whole grid runs longest-first.
+  const int qb = static_cast<int>(gridDim.y) - 1 - static_cast<int>(blockIdx.y);
 
   // ---- block-uniform work description (identical in every thread) ---------
   const int32_t p = a.prefix_lens[r];
   const int64_t qbase = a.q_offsets[r];
   const int32_t e = a.prefix_mode ? static_cast<int32_t>(a.q_offsets[r + 1] - qbase) : a.extend_lens[r];
   if (p < 0 || e < 0 || qbase < 0 || qbase + e > a.total_q) {
-    if (threadIdx.x == 0 && blockIdx.x == 0 && g == 0) set_err(a.err, PKV_DEV_ERR_BAD_LENGTH);
+    if (threadIdx.x == 0 && blockIdx.y == 0 && g == 0) set_err(a.err, PKV_DEV_ERR_BAD_LENGTH);
     return;
   }
-  if (e > a.max_extend && threadIdx.x == 0 && blockIdx.x == 0 && g == 0)
+  if (e > a.max_extend && threadIdx.x == 0 && blockIdx.y == 0 && g == 0)
     set_err(a.err, PKV_DEV_ERR_BAD_LENGTH);
   const int i0 = qb * (kQTiles * TQ);
   if (i0 >= e) return;
@@ -706,7 +713,8 @@ cudaError_t launch_g(const CUtensorMap& qm, const ExtendTcArgs& a,
   cudaError_t e = ensure_smem_limit(extend_tc_kernel<G>, kSmemBytes, smem_state);
   if (e != cudaSuccess) return e;
   if (grid_z > 65535) return cudaErrorInvalidValue;
-  dim3 grid(nqb, a.hkv, static_cast<unsigned>(grid_z));
+  if (nqb > 65535) return cudaErrorInvalidValue;
+  dim3 grid(a.hkv, nqb, static_cast<unsigned>(grid_z));
   extend_tc_kernel<G><<<grid, kThreads, kSmemBytes, s>>>(qm, a);
   return cudaGetLastError();
 }
