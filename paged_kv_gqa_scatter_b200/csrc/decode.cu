@@ -173,6 +173,11 @@ __global__ void __launch_bounds__(32 * 9, 1) decode_split_kernel(const DecodeArg
     fence_barrier_init();
   }
 
+  // Every input (lengths, table rows, page table, pool) may come from the
+  // preceding kernel on the stream: wait for it before reading any of them.
+  // Launch and the barrier set-up above still overlap its tail.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+
   // ---- plan: prefix sums of clamped context lengths -------------------------
   // One warp: each lane sums a contiguous segment of requests, one shuffle
   // scan combines the segments, and each lane writes its segment's prefixes.
@@ -285,8 +290,6 @@ __global__ void __launch_bounds__(32 * 9, 1) decode_split_kernel(const DecodeArg
     int32_t e1 = lookup(c1, h1);
     c2 = c1;
     bool h2 = h1 && advance(c2);
-    // Rows written by the preceding store_kv must be visible before any copy.
-    asm volatile("griddepcontrol.wait;" ::: "memory");
     int last_use[kStages];
 #pragma unroll
     for (int i = 0; i < kStages; ++i) last_use[i] = -1;
@@ -626,11 +629,11 @@ cudaError_t launch_decode_t(const DecodeArgs& a, int grid, cudaStream_t s, const
   if (L.total > max_bytes) return cudaErrorInvalidValue;
   cudaError_t e = ensure_smem_limit(decode_split_kernel<E, G>, max_bytes, smem_state);
   if (e != cudaSuccess) return e;
-  // Both kernels use programmatic dependent launch: the split kernel's set-up
-  // (barriers, length scan, first table reads) overlaps the tail of the
-  // preceding kernel and waits (griddepcontrol.wait) before reading the pool;
-  // the combine kernel is scheduled while the split kernel runs and waits
-  // for its partials.
+  // Both kernels use programmatic dependent launch: the split kernel is
+  // scheduled and sets up its barriers while the preceding kernel finishes,
+  // and reads nothing (lengths, table, pool) before griddepcontrol.wait; the
+  // combine kernel is scheduled while the split kernel runs and waits for
+  // its partials.
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;

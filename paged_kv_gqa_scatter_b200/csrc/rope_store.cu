@@ -103,6 +103,9 @@ template <typename E, int kThreads, int kRif, int kMinBlocks, bool kFp8>
 __global__ void __launch_bounds__(kThreads, kMinBlocks) qk_norm_rope_store_kernel(const RopeArgs a) {
   constexpr int kPoolEsize = kFp8 ? 1 : static_cast<int>(sizeof(E));
   constexpr int kHalfWarps = kThreads / 16;
+  // An attention kernel launched next may be scheduled now; it waits for
+  // this grid before it reads anything.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int64_t t = blockIdx.x;
   const int rows = a.hq + 2 * a.hkv;
   const int hw = threadIdx.x >> 4;  // half-warp: the first row it owns
