@@ -63,3 +63,51 @@ def test_bf16_rounding_ties_to_even():
     back = W.bf16_bits_to_f32(bits)
     # 1 + 2^-8 is a tie between 1 and 1 + 2^-7 -> even (1.0); 1 + 3*2^-8 -> 1 + 2^-6.
     assert back.tolist() == [1.0, 1.0, 1.0 + 2 ** -6, -2.5, 65536.0]
+
+
+def test_grouped_decode_structure():
+    """Members of a group share the prefix slots; suffix slots are private and
+    distinct; every context covers its group's prefix plus the stored token."""
+    for P in (1, 16, 64):
+        gd = W.grouped_decode(page_size=P)
+        d = gd.decode
+        off, plen = gd.group_offsets, gd.group_prefix_lens
+        assert off[0] == 0 and off[-1] == d.batch and np.all(np.diff(off) >= 1)
+        seen = []
+        for g in range(len(plen)):
+            rows = [d.table_idx[r] for r in range(off[g], off[g + 1])]
+            p = int(plen[g])
+            for r, row in zip(range(off[g], off[g + 1]), rows):
+                assert np.array_equal(d.page_table[row, :p], d.page_table[rows[0], :p])
+                assert d.seq_lens[r] >= p + 1
+                seen.append(d.page_table[row, p:d.seq_lens[r]])
+            seen.append(d.page_table[rows[0], :p])
+        allslots = np.concatenate(seen)
+        assert len(np.unique(allslots)) == len(allslots)
+        assert np.all(allslots < d.pool.num_slots)
+        if P > 1:
+            assert np.all(plen % P == 0)
+
+
+def test_fp8_pool_variant():
+    base = W.decode_small()
+    wl = W.with_fp8_pool(base)
+    assert wl.pool.dtype == W.F8 and wl.pool.io_dtype == W.BF16
+    assert wl.k_planes[0].dtype == np.uint8 and wl.k_planes[0].shape == base.k_planes[0].shape
+    codes = wl.k_planes[0]
+    assert not np.any((codes & 0x7F) == 0x7F)                 # no NaN codes
+    ex = (codes >> 3) & 0xF
+    assert ex.min() >= 4 and ex.max() <= 9
+    assert np.array_equal(wl.q, base.q) and np.array_equal(wl.k_new, base.k_new)
+    assert wl.pool.k_scale == float(np.float32(0.05))
+
+
+def test_rope_store_step_inputs():
+    wl = W.rope_store_step()
+    assert wl.qkv.shape == (wl.n_tokens, (wl.num_q_heads + 2 * wl.pool.num_kv_heads) * W.HEAD_DIM)
+    assert np.all((wl.positions >= 0) & (wl.positions < wl.cos_sin_cache.shape[0]))
+    assert len(np.unique(wl.out_loc)) == wl.n_tokens
+    cs = wl.cos_sin_cache.astype(np.float64)
+    # cos^2 + sin^2 = 1 for every stored angle (float32 table).
+    assert np.allclose(cs[:, :64] ** 2 + cs[:, 64:] ** 2, 1.0, atol=1e-6)
+    assert np.array_equal(cs[0, :64], np.ones(64)) and np.array_equal(cs[0, 64:], np.zeros(64))
