@@ -304,9 +304,8 @@ def run_decode(args, world, rank, local):
         step()
     torch.cuda.synchronize()
 
-    # ---- timed region: K steps, events per call on the launching stream ------
+    # ---- timed region: exactly K steps, launched back to back ----------------
     nL = len(layers)
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps * nL)]
     start = torch.cuda.Event(enable_timing=True)
     stop = torch.cuda.Event(enable_timing=True)
     clocks = ClockSampler(local)
@@ -314,6 +313,19 @@ def run_decode(args, world, rank, local):
     torch.cuda.synchronize()
     clocks.start()
     start.record(stream)
+    for _ in range(args.steps):
+        step()
+    stop.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    ms_total = start.elapsed_time(stop)
+    ms_total = max_over_ranks(ms_total, world)
+
+    # ---- per-call durations for the roofline: K more steps, events around
+    # each call on the launching stream (the events cost the calls their
+    # launch overlap, so this loop is not the one `value` comes from) -------
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps * nL)]
     i = 0
     for _ in range(args.steps):
         for l in layers:
@@ -323,12 +335,7 @@ def run_decode(args, world, rank, local):
             api.decode_attn(pool, l, q, table, table_idx, seq_lens, out, ws, scale=wl.scale, dev_err=err)
             ev[i][2].record(stream)
             i += 1
-    stop.record(stream)
     torch.cuda.synchronize()
-    barrier(world)
-    clk = clocks.stop()
-    ms_total = start.elapsed_time(stop)
-    ms_total = max_over_ranks(ms_total, world)
     dec_ms = [e[1].elapsed_time(e[2]) for e in ev]
     st_ms = [e[0].elapsed_time(e[1]) for e in ev]
     errv = int(err.item())
@@ -358,11 +365,28 @@ def run_decode(args, world, rank, local):
     # an upload stream while step k computes, and step k's output is read
     # back on a download stream.  Every step's inputs are copied and its
     # output read inside the timed region.
+    # The step's inputs travel as one packed buffer (one copy per step): q,
+    # k_new, v_new, out_loc, seq_lens, table_idx and the page table, each at
+    # a 256-byte aligned offset; the device side takes typed views of it.
+    parts = [("q", h_q, q), ("k", h_k, k_new), ("v", h_v, v_new), ("loc", h_loc, out_loc),
+             ("sl", h_sl, seq_lens), ("ti", h_ti, table_idx), ("pt", h_pt, table.entries)]
+    offs, total_b = {}, 0
+    for name, h, _ in parts:
+        offs[name] = total_b
+        total_b += (h.numel() * h.element_size() + 255) // 256 * 256
+    h_pack = _t.empty(total_b, dtype=_t.uint8).pin_memory()
+    for name, h, _ in parts:
+        nb = h.numel() * h.element_size()
+        h_pack[offs[name]:offs[name] + nb].copy_(h.reshape(-1).view(_t.uint8))
+
+    h2d = total_b  # the bytes actually copied per step (with alignment padding)
+
     def dev_set():
-        d = {"q": torch.empty_like(q), "k": torch.empty_like(k_new), "v": torch.empty_like(v_new),
-             "loc": torch.empty_like(out_loc), "sl": torch.empty_like(seq_lens),
-             "ti": torch.empty_like(table_idx), "pt": torch.empty_like(table.entries),
-             "out": torch.empty_like(out)}
+        buf = torch.empty(total_b, dtype=torch.uint8, device=dev)
+        d = {"buf": buf, "out": torch.empty_like(out)}
+        for name, h, like in parts:
+            nb = h.numel() * h.element_size()
+            d[name] = buf[offs[name]:offs[name] + nb].view(like.dtype).view(like.shape)
         d["table"] = api.PageTable(d["pt"])
         return d
 
@@ -376,13 +400,7 @@ def run_decode(args, world, rank, local):
         d = sets[bi]
         up.wait_event(comp_done[bi])  # the set's previous step has finished with it
         with torch.cuda.stream(up):
-            d["q"].view(_t.int16).copy_(h_q, non_blocking=True)
-            d["k"].view(_t.int16).copy_(h_k, non_blocking=True)
-            d["v"].view(_t.int16).copy_(h_v, non_blocking=True)
-            d["loc"].copy_(h_loc, non_blocking=True)
-            d["sl"].copy_(h_sl, non_blocking=True)
-            d["ti"].copy_(h_ti, non_blocking=True)
-            d["pt"].copy_(h_pt, non_blocking=True)
+            d["buf"].copy_(h_pack, non_blocking=True)
         up_done[bi].record(up)
 
     def e2e_run(nsteps):
@@ -484,7 +502,7 @@ def run_decode(args, world, rank, local):
             "algorithmic_bytes_per_launch": per_call,
         },
         "e2e": {"value": round(e2e_val, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
-                "pipeline": "step k+1's host->device copies overlap step k; read-back on its own stream",
+                "pipeline": "one packed host->device copy per step; step k+1's copy overlaps step k; read-back on its own stream",
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": 3 * args.steps * nL,
         "device_error_word": errv,

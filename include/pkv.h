@@ -200,6 +200,19 @@ int pkv_qk_norm_rope_store(const pkv_pool* pool, int32_t layer, const void* qkv,
                            int32_t* dev_err, pkv_stream_t stream);
 
 /*
+ * selftest_wait_timeout -- exercises the bounded wait of the pipelined
+ * kernels.  The pages have no counterpart; it exists so that a test can
+ * check, without faulting anything, that a wait nobody satisfies gives up.
+ *
+ * Launches one 32-thread kernel that waits on a shared-memory mbarrier that
+ * nothing signals, with the same wait routine decode and extend use.  After
+ * about one second the wait gives up, PKV_DEV_ERR_TIMEOUT is OR-ed into
+ * *dev_err (device int32, required), and the kernel returns; the stream and
+ * context remain usable.  Asynchronous like every other call.
+ */
+int pkv_selftest_wait_timeout(int32_t* dev_err, pkv_stream_t stream);
+
+/*
  * gather_kv -- copies requests' K/V rows, in token order, through the page
  * table into dense buffers [P5 §4.6.4 page-table translation].  It is the
  * translation step the attention kernels perform internally, exposed on its

@@ -40,6 +40,7 @@ SIGNATURES = {
     "pkv_qk_norm_rope_store": (ctypes.c_int, [ctypes.POINTER(PkvPool), c_i32, c_vp, c_i64, c_i32, c_vp,
                                               c_i32, c_vp, c_i64, c_vp, c_vp, ctypes.c_float, c_vp,
                                               c_i32, c_i64, c_vp, c_vp, c_vp]),
+    "pkv_selftest_wait_timeout": (ctypes.c_int, [c_vp, c_vp]),
     "pkv_gather_kv": (ctypes.c_int, [ctypes.POINTER(PkvPool), c_i32, ctypes.POINTER(PkvPageTable),
                                      c_vp, c_vp, c_vp, c_i32, c_vp, c_vp, c_vp, c_vp]),
     "pkv_decode_workspace_bytes": (c_size, [c_i32, c_i32]),

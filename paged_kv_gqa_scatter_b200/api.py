@@ -144,6 +144,14 @@ def qk_norm_rope_store(pool: KVPool, layer: int, qkv: torch.Tensor, num_q_heads:
         q_out.data_ptr(), _ptr(dev_err), _stream_ptr(stream)), "qk_norm_rope_store")
 
 
+def selftest_wait_timeout(dev_err: torch.Tensor, stream=None) -> None:
+    """pkv_selftest_wait_timeout: a kernel whose barrier wait must give up
+    after about one second and set DEV_ERR_TIMEOUT in dev_err."""
+    _require_cuda(dev_err)
+    _lib.check(_lib.load().pkv_selftest_wait_timeout(dev_err.data_ptr(), _stream_ptr(stream)),
+               "selftest_wait_timeout")
+
+
 def gather_kv(pool: KVPool, layer: int, table: PageTable, table_idx: torch.Tensor,
               seq_lens: torch.Tensor, row_offsets: torch.Tensor, k_out: torch.Tensor,
               v_out: torch.Tensor, dev_err: Optional[torch.Tensor] = None, stream=None) -> None:

@@ -156,6 +156,11 @@ int pkv_qk_norm_rope_store(const pkv_pool* pool, int32_t layer, const void* qkv,
       q_out, dev_err, static_cast<cudaStream_t>(stream)));
 }
 
+int pkv_selftest_wait_timeout(int32_t* dev_err, pkv_stream_t stream) {
+  if (dev_err == nullptr) return PKV_ERR_INVALID_ARG;
+  return from_cuda(pkv::launch_wait_timeout(dev_err, static_cast<cudaStream_t>(stream)));
+}
+
 int pkv_gather_kv(const pkv_pool* pool, int32_t layer, const pkv_page_table* table,
                   const int32_t* table_idx, const int32_t* seq_lens, const int64_t* row_offsets,
                   int32_t batch, void* k_out, void* v_out, int32_t* dev_err,

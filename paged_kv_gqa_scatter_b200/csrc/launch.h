@@ -59,6 +59,8 @@ cudaError_t launch_qk_norm_rope_store(const PoolView& pool, const void* qkv, int
                                       const void* k_w, float eps, const void* out_loc, bool loc_i64,
                                       int64_t n, void* q_out, int32_t* err, cudaStream_t s);
 
+cudaError_t launch_wait_timeout(int32_t* err, cudaStream_t s);
+
 cudaError_t launch_gather_kv(const PoolView& pool, const TableView& t, const int32_t* table_idx,
                              const int32_t* seq_lens, const int64_t* row_offsets, int32_t batch,
                              void* k_out, void* v_out, int32_t* err, cudaStream_t s);
