@@ -243,9 +243,12 @@ def run_decode(args, world, rank, local):
     torch.cuda.set_device(dev)
     if args.workload == "decode-qwen3-8b":
         free, _ = torch.cuda.mem_get_info()
-        bytes_per_page = 36 * 16 * 8 * 128 * 2 * 2
+        P = args.page_size or 16
+        bytes_per_page = 36 * P * 8 * 128 * 2 * 2
         num_pages = int(0.6 * free // bytes_per_page)
-        wl = W.decode_qwen3_8b(num_pages=num_pages)
+        wl = W.decode_qwen3_8b(num_pages=num_pages, page_size=P)
+        if P != 16:
+            wl.name = f"decode-qwen3-8b-p{P}"
         layers = list(range(wl.pool.num_layers))
     else:
         nl = 28 if args.pool_layers is None else args.pool_layers
@@ -951,6 +954,8 @@ def main():
     ap.add_argument("--pool-layers", type=int, default=None,
                     help="pool layers of decode-qwen3-0.6b (28) or radix-prefix (32); fewer only for profiling")
     ap.add_argument("--no-extend", action="store_true")
+    ap.add_argument("--page-size", type=int, default=None,
+                    help="page size of decode-qwen3-8b (16 as stated; 64 is TRT-LLM's size)")
     ap.add_argument("--kv-dtype", choices=["bf16", "fp8"], default="bf16",
                     help="pool element type of decode-qwen3-0.6b (fp8: scaled E4M3 codes, bf16 q/out)")
     ap.add_argument("--radix-decode", choices=["cascade", "plain"], default="cascade",
