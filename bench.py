@@ -518,9 +518,10 @@ def run_decode(args, world, rank, local):
         gbs, sample, _ = cpu_decode_sample(wl)
         result["cpu_baseline"] = {"value": round(gbs, 4), "unit": "GB/s", "cores": blas_threads(),
                                   "kind": "oracle", "sample": sample}
-    if not args.no_extend and args.workload == "decode-qwen3-0.6b" and not fp8:
-        result["extend"] = run_extend_measure(dev, warmup=3, iters=max(5, args.steps))
-        result["qk_norm_rope_store"] = run_rope_measure(dev, iters=max(5, args.steps))
+    if not args.no_extend and args.workload == "decode-qwen3-0.6b":
+        result["extend"] = run_extend_measure(dev, warmup=3, iters=max(5, args.steps), fp8=fp8)
+        if not fp8:
+            result["qk_norm_rope_store"] = run_rope_measure(dev, iters=max(5, args.steps))
     return result
 
 
@@ -588,22 +589,30 @@ def run_rope_measure(dev, iters=10, warmup=3):
     return out
 
 
-def run_extend_measure(dev, warmup=3, iters=10):
+def run_extend_measure(dev, warmup=3, iters=10, fp8=False):
     """Extend TFLOP/s on the chunked-prefill step (2048-token chunk at prefix 6144,
-    Hq 32, Hkv 8): causal FLOPs = 4 d Hq (e p + e (e+1) / 2)."""
+    Hq 32, Hkv 8): causal FLOPs = 4 d Hq (e p + e (e+1) / 2).  fp8: the same
+    chunk over an E4M3 copy of the pool."""
     import torch
     from paged_kv_gqa_scatter_b200 import api
     from paged_kv_gqa_scatter_b200 import workloads as W
     mix = W.chunked_prefill_step(step=3)
-    wl = mix.extend
+    wl = W.with_fp8_pool(mix.extend) if fp8 else mix.extend
 
     def tdev(a):
         return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
 
+    def tpool(a):
+        if fp8:
+            return torch.from_numpy(np.ascontiguousarray(a)).to(dev).view(torch.float8_e4m3fn)
+        return tdev(a)
+
     spec = wl.pool
-    pool = api.KVPool.empty(spec.num_layers, spec.num_slots, spec.num_kv_heads, device=dev)
-    pool.k[0].copy_(tdev(wl.k_planes[0]))
-    pool.v[0].copy_(tdev(wl.v_planes[0]))
+    pool = api.KVPool.empty(spec.num_layers, spec.num_slots, spec.num_kv_heads, device=dev,
+                            dtype=torch.float8_e4m3fn if fp8 else torch.bfloat16,
+                            k_scale=spec.k_scale, v_scale=spec.v_scale)
+    pool.k[0].copy_(tpool(wl.k_planes[0]))
+    pool.v[0].copy_(tpool(wl.v_planes[0]))
     table = api.PageTable(torch.from_numpy(wl.page_table).to(dev))
     ti = torch.from_numpy(wl.table_idx).to(dev)
     pl = torch.from_numpy(wl.prefix_lens).to(dev)
@@ -629,13 +638,14 @@ def run_extend_measure(dev, warmup=3, iters=10):
     flops = 4 * 128 * wl.num_q_heads * wl.causal_pairs()
     _, bf16, _, src = measured_peaks()
     tf = flops / (med / 1e3) / 1e12
-    return {"workload": "chunked-prefill extend, 2048-token chunk at prefix 6144, Hq 32 Hkv 8",
+    return {"workload": "chunked-prefill extend, 2048-token chunk at prefix 6144, Hq 32 Hkv 8"
+                        + (", E4M3 pool" if fp8 else ""),
             "tflops": round(tf, 2), "ms": round(med, 4), "flops": flops,
             "roofline": {"bound": "tensor", "achieved": round(tf, 2), "peak": bf16,
                          "peak_source": src, "unit": "TFLOP/s", "frac": round(tf / bf16, 4),
-                         "traffic": recorded_traffic("extend_tc_kernel",
-                                                     source_hash("extend_tc.cu", "common.cuh"),
-                                                     "chunked-prefill extend c3")},
+                         "traffic": None if fp8 else recorded_traffic("extend_tc_kernel",
+                                                                      source_hash("extend_tc.cu", "common.cuh"),
+                                                                      "chunked-prefill extend c3")},
             "device_error_word": int(err.item())}
 
 

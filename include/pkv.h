@@ -91,10 +91,10 @@ typedef enum { PKV_DTYPE_BF16 = 0, PKV_DTYPE_F32 = 1, PKV_DTYPE_FP8_E4M3 = 2 } p
  * the model dtype): each plane element is an OCP E4M3 code (1 byte) standing
  * for code_value * k_scale (K plane) or * v_scale (V plane).  Calls that
  * write the pool take bf16 rows and store the code of x * (1 / scale)
- * (float32 product, round to nearest even, saturated to +-448); decode reads
- * the codes and takes q and returns out in bf16.  Extend and cascade decode
- * return PKV_ERR_UNSUPPORTED for FP8 pools.  The scales must be finite and
- * > 0; they are ignored for the other dtypes.
+ * (float32 product, round to nearest even, saturated to +-448); decode,
+ * cascade decode and extend read the codes (extend widens them to f16 for
+ * the tensor cores) and take q and return out in bf16.  The scales must be
+ * finite and > 0; they are ignored for the other dtypes.
  */
 typedef struct {
   void* k;
@@ -320,7 +320,7 @@ int pkv_decode_attn_noalloc(const pkv_pool* pool, int32_t layer, const void* q,
  *   finite.
  * workspace: pkv_decode_cascade_workspace_bytes(batch, num_q_heads,
  *   max_prefix_len) bytes, 16-byte aligned.
- * bf16 pools only (PKV_ERR_UNSUPPORTED otherwise); other limits as
+ * bf16 and FP8 pools (PKV_ERR_UNSUPPORTED for fp32); other limits as
  * decode_attn.
  */
 size_t pkv_decode_cascade_workspace_bytes(int32_t batch, int32_t num_q_heads,

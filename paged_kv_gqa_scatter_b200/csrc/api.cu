@@ -229,7 +229,7 @@ int pkv_decode_attn_cascade(const pkv_pool* pool, int32_t layer, const void* q,
   TableView tv;
   int st = check_pool(pool, layer, &pv);
   if (st != PKV_OK) return st;
-  if (pv.dtype != PKV_DTYPE_BF16) return PKV_ERR_UNSUPPORTED;
+  if (pv.dtype == PKV_DTYPE_F32) return PKV_ERR_UNSUPPORTED;
   st = check_heads(pool, num_q_heads);
   if (st != PKV_OK) return st;
   if (batch < 0 || num_groups < 0 || max_prefix_len < 0) return PKV_ERR_INVALID_ARG;
@@ -279,9 +279,8 @@ int pkv_extend_attn(const pkv_pool* pool, int32_t layer, const void* q, int32_t 
   if (!q || !out || !table_idx || !prefix_lens || !extend_lens || !q_offsets)
     return PKV_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(out)) return PKV_ERR_MISALIGNED;
-  if (pv.dtype == PKV_DTYPE_FP8_E4M3) return PKV_ERR_UNSUPPORTED;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (pv.dtype == PKV_DTYPE_BF16)
+  if (pv.dtype == PKV_DTYPE_BF16 || pv.dtype == PKV_DTYPE_FP8_E4M3)
     return from_cuda(pkv::launch_extend_tc(pv, tv, q, num_q_heads, table_idx, prefix_lens,
                                            extend_lens, q_offsets, batch, total_q, max_extend_len, scale,
                                            out, dev_err, s));

@@ -88,6 +88,7 @@ constexpr int kBarSFull = 17;   // + 2 * q tile + half
 constexpr int kBarPReady = 21;  // + 2 * q tile + half
 constexpr int kBarODone = 25;   // + q tile
 constexpr int kBarOFinal = 27;
+constexpr int kBarQReady = 28;  // FP8 pools: Q converted to f16 in place
 
 // TMEM columns: S_i (two 64-column halves, one per step parity) and O_i.
 constexpr uint32_t kTmemCols = 512;
@@ -126,6 +127,7 @@ struct ExtendTcArgs {
   int32_t nreq;    // query rows (requests) in q
   float2* pre_ml;  // [nsplit][nreq][hq]
   float* pre_o;    // [nsplit][nreq][hq][128]
+  float v_scale;   // FP8 pools: V dequantisation scale (1 otherwise)
 };
 
 // ---- PTX wrappers -----------------------------------------------------------
@@ -156,10 +158,35 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint3
   return d;
 }
 
-// Instruction descriptors, kind::f16: bf16 A/B, fp32 D, M = 128.
+// Instruction descriptors, kind::f16: bf16 A/B (f16 A/B for FP8 pools, whose
+// codes widen exactly to f16), fp32 D, M = 128.
 constexpr uint32_t kIdescF16 = (1u << 4) | (1u << 7) | (1u << 10) | ((128u >> 4) << 24);
+constexpr uint32_t kIdescHalf = (1u << 4) | ((128u >> 4) << 24);
 constexpr uint32_t kIdescQK = kIdescF16 | ((64u >> 3) << 17);                // N = 64 keys, A and B K-major
 constexpr uint32_t kIdescPV = kIdescF16 | ((128u >> 3) << 17) | (1u << 16);  // N = 128 dims, B (V) MN-major
+constexpr uint32_t kIdescQKHalf = kIdescHalf | ((64u >> 3) << 17);
+constexpr uint32_t kIdescPVHalf = kIdescHalf | ((128u >> 3) << 17) | (1u << 16);
+
+// Two floats -> f16x2 (round to nearest even), a in the low half.
+__device__ __forceinline__ uint32_t pack_f16x2(float a, float b) {
+  __half2 h = __floats2half2_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// 16 E4M3 codes -> 16 f16 values (exact), as two 16-byte words.
+__device__ __forceinline__ void e4m3x16_to_f16(const uint4& w, uint4& lo, uint4& hi) {
+  const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+  uint32_t o[8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const __half2_raw a = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(u[i] & 0xffffu), __NV_E4M3);
+    const __half2_raw b = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(u[i] >> 16), __NV_E4M3);
+    o[2 * i] = static_cast<uint32_t>(a.x) | (static_cast<uint32_t>(a.y) << 16);
+    o[2 * i + 1] = static_cast<uint32_t>(b.x) | (static_cast<uint32_t>(b.y) << 16);
+  }
+  lo = make_uint4(o[0], o[1], o[2], o[3]);
+  hi = make_uint4(o[4], o[5], o[6], o[7]);
+}
 
 __device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                        uint32_t accum) {
@@ -274,9 +301,15 @@ __device__ __forceinline__ bool elect_one() {
 }
 
 // ---- the kernel ---------------------------------------------------------------
-template <int G>
+// kFp8: the pool holds E4M3 codes.  The load warps widen each K/V row to f16
+// on the way into shared memory, the softmax warps convert the bf16 Q tiles
+// to f16 in place, and the MMAs run on f16 operands (P is packed as f16).
+template <int G, bool kFp8>
 __global__ void __launch_bounds__(kThreads, 1)
     extend_tc_kernel(const __grid_constant__ CUtensorMap qmap, const ExtendTcArgs a) {
+  constexpr uint32_t kIdQK = kFp8 ? kIdescQKHalf : kIdescQK;
+  constexpr uint32_t kIdPV = kFp8 ? kIdescPVHalf : kIdescPV;
+  constexpr int kRowBytes = kFp8 ? 128 : 256;  // one KV head of one slot in the pool
   constexpr int TQ = kRowsPerTile / G;  // tokens per Q tile
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -345,6 +378,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < kQTiles; ++i) mbar_init(&bars[kBarODone + i], 1);
     mbar_init(&bars[kBarOFinal], 1);
+    mbar_init(&bars[kBarQReady], 2 * 128);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -401,12 +435,39 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int t = 0; t < 16; ++t) {
           const int kk = u * 32 + 2 * t + h;  // key within the step
           const int32_t slot = __shfl_sync(0xffffffffu, sl[u], 2 * t + h);
-          const uint8_t* src = base + static_cast<int64_t>(slot) * a.slot_stride_bytes + g * 256 + c * 16;
+          const uint8_t* src = base + static_cast<int64_t>(slot) * a.slot_stride_bytes + g * kRowBytes + c * 16;
           const uint32_t dst = dst_tile + (c >> 3) * kKvHalfBytes + kk * 128 + (((c & 7) ^ (kk & 7)) << 4);
           asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
         }
       }
       asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+    // FP8: 8 lanes per key row (16 codes each, one 16-byte load), 4 rows per
+    // instruction; every load of the step is issued before the first
+    // conversion, and each 16-code chunk becomes two f16 chunks of the same
+    // swizzled layout, stored with plain shared-memory stores.
+    auto copy_step_f8 = [&](const uint8_t* base, uint8_t* dst_tile, const int32_t (&sl)[2]) {
+      const int q4 = lane >> 3, cf = lane & 7;
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {  // keys u*32 .. u*32 + 31: 8 loads in flight per lane
+        uint4 raw[8];
+#pragma unroll
+        for (int it = 0; it < 8; ++it) {
+          const int kk = u * 32 + it * 4 + q4;
+          const int32_t slot = __shfl_sync(0xffffffffu, sl[u], kk & 31);
+          raw[it] = __ldg(reinterpret_cast<const uint4*>(base + static_cast<int64_t>(slot) * a.slot_stride_bytes +
+                                                         g * kRowBytes + cf * 16));
+        }
+#pragma unroll
+        for (int it = 0; it < 8; ++it) {
+          const int kk = u * 32 + it * 4 + q4;
+          uint4 lo, hi;
+          e4m3x16_to_f16(raw[it], lo, hi);
+          const int c0 = 2 * cf, c1 = 2 * cf + 1;
+          *reinterpret_cast<uint4*>(dst_tile + (c0 >> 3) * kKvHalfBytes + kk * 128 + (((c0 & 7) ^ (kk & 7)) << 4)) = lo;
+          *reinterpret_cast<uint4*>(dst_tile + (c1 >> 3) * kKvHalfBytes + kk * 128 + (((c1 & 7) ^ (kk & 7)) << 4)) = hi;
+        }
+      }
     };
     int32_t sl[2];
     lookup(par, sl);
@@ -421,17 +482,27 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
       }
-      // K and V copies of the step fly together; K is signalled first.
-      copy_step(a.kbase, smem_u32(sK + st * kKvTileBytes), sl);
-      copy_step(a.vbase, smem_u32(sV + st * kKvTileBytes), sl);
       int32_t nsl[2];
-      lookup(j + 2, nsl);  // this warp's next step; the loads fly with the copies
-      asm volatile("cp.async.wait_group 1;" ::: "memory");
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      mbar_arrive(&bars[kBarKFull + st]);
-      asm volatile("cp.async.wait_group 0;" ::: "memory");
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      mbar_arrive(&bars[kBarVFull + st]);
+      if constexpr (kFp8) {
+        copy_step_f8(a.kbase, sK + st * kKvTileBytes, sl);
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        mbar_arrive(&bars[kBarKFull + st]);
+        lookup(j + 2, nsl);
+        copy_step_f8(a.vbase, sV + st * kKvTileBytes, sl);
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        mbar_arrive(&bars[kBarVFull + st]);
+      } else {
+        // K and V copies of the step fly together; K is signalled first.
+        copy_step(a.kbase, smem_u32(sK + st * kKvTileBytes), sl);
+        copy_step(a.vbase, smem_u32(sV + st * kKvTileBytes), sl);
+        lookup(j + 2, nsl);  // this warp's next step; the loads fly with the copies
+        asm volatile("cp.async.wait_group 1;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        mbar_arrive(&bars[kBarKFull + st]);
+        asm volatile("cp.async.wait_group 0;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        mbar_arrive(&bars[kBarVFull + st]);
+      }
       sl[0] = nsl[0];
       sl[1] = nsl[1];
     }
@@ -467,7 +538,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kk = 0; kk < 8; ++kk) {
           const uint64_t ao = static_cast<uint64_t>(((kk >> 2) * kQHalfBytes + (kk & 3) * 32) >> 4);
           const uint64_t bo = static_cast<uint64_t>(((kk >> 2) * kKvHalfBytes + (kk & 3) * 32) >> 4);
-          mma_ss(d, ad + ao, bd + bo, kIdescQK, kk > 0 ? 1u : 0u);
+          mma_ss(d, ad + ao, bd + bo, kIdQK, kk > 0 ? 1u : 0u);
         }
         mma_commit(&bars[kBarSFull + 2 * i + (j & 1)]);
       }
@@ -480,7 +551,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (elect_one()) {
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          mma_ts(d, pa + kk * 8, bd + static_cast<uint64_t>((kk * 2048) >> 4), kIdescPV,
+          mma_ts(d, pa + kk * 8, bd + static_cast<uint64_t>((kk * 2048) >> 4), kIdPV,
                  (j == 0 && kk == 0) ? 0u : 1u);
         mma_commit(&bars[kBarODone + i]);
       }
@@ -493,7 +564,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto wait_all = [&](int bar, uint32_t parity) -> bool {
       return __all_sync(0xffffffffu, mbar_wait(&bars[bar], parity));
     };
-    bool ok = wait_all(kBarQFull, 0);
+    bool ok = wait_all(kFp8 ? kBarQReady : kBarQFull, 0);
     for (int j = 0; j < 2 && j < nsteps && ok; ++j) {
       ok = wait_all(kBarKFull + j, 0);
       if (!ok) break;
@@ -549,6 +620,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     float2 l2 = make_float2(0.f, 0.f);  // running sum of p, even / odd keys
     const float2 sl2 = make_float2(a.scale_log2, a.scale_log2);
     bool ok = true;
+    if constexpr (kFp8) {
+      // Convert both Q tiles from bf16 to f16 in place (the swizzle permutes
+      // whole 16-byte chunks, so each chunk is converted where it lies), make
+      // the stores visible to the tensor core, then release the MMA warp.
+      const bool wq = mbar_wait(&bars[kBarQFull], 0);
+      if (__any_sync(0xffffffffu, !wq)) ok = false;
+      uint4* qc = reinterpret_cast<uint4*>(sQ);
+      constexpr int kChunks = kQTiles * kQTileBytes / 16;
+#pragma unroll 4
+      for (int k = threadIdx.x; k < kChunks; k += 2 * 128) {
+        const uint4 w = qc[k];
+        const float2 f0 = bf16x2_to_f2(w.x), f1 = bf16x2_to_f2(w.y), f2 = bf16x2_to_f2(w.z), f3 = bf16x2_to_f2(w.w);
+        qc[k] = make_uint4(pack_f16x2(f0.x, f0.y), pack_f16x2(f1.x, f1.y), pack_f16x2(f2.x, f2.y),
+                           pack_f16x2(f3.x, f3.y));
+      }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      mbar_arrive(&bars[kBarQReady]);
+    }
     for (int j = 0; j < nsteps; ++j) {
       const int hf = j & 1;
       const uint32_t s_addr = tmem + lane_base + kColS + 128 * i + 64 * hf;
@@ -604,7 +693,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                         sl2, negm2);
             const float2 pp = make_float2(ex2_approx(t.x), ex2_approx(t.y));
             l2 = __fadd2_rn(l2, pp);
-            w16[u >> 1] = pack_bf16x2(pp.x, pp.y);
+            w16[u >> 1] = kFp8 ? pack_f16x2(pp.x, pp.y) : pack_bf16x2(pp.x, pp.y);
           }
         } else {
 #pragma unroll
@@ -614,7 +703,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float p0 = (32 * c + u < vis) ? ex2_approx(t.x) : 0.f;
             const float p1 = (32 * c + u + 1 < vis) ? ex2_approx(t.y) : 0.f;
             l2 = __fadd2_rn(l2, make_float2(p0, p1));
-            w16[u >> 1] = pack_bf16x2(p0, p1);
+            w16[u >> 1] = kFp8 ? pack_f16x2(p0, p1) : pack_bf16x2(p0, p1);
           }
         }
         tmem_st16(s_addr + 16 * c, w16);
@@ -640,13 +729,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(o_addr + c * 32, o);
         if (valid) {
 #pragma unroll
-          for (int u = 0; u < 32; u += 4)
-            *reinterpret_cast<float4*>(dst + c * 32 + u) = make_float4(o[u], o[u + 1], o[u + 2], o[u + 3]);
+          for (int u = 0; u < 32; u += 4) {
+            const float vs = kFp8 ? a.v_scale : 1.f;
+            *reinterpret_cast<float4*>(dst + c * 32 + u) =
+                make_float4(o[u] * vs, o[u + 1] * vs, o[u + 2] * vs, o[u + 3] * vs);
+          }
         }
       }
       if (valid) a.pre_ml[row] = make_float2(m_run, l_run);
     } else if (w && ok) {
-      const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+      const float inv = (l_run > 0.f ? 1.f / l_run : 0.f) * (kFp8 ? a.v_scale : 1.f);
       __nv_bfloat16* dst = a.out + ((qbase + tok) * a.hq + g * G + hh) * kHeadDim;
 #pragma unroll 1
       for (int c = 0; c < 4; ++c) {
@@ -704,19 +796,37 @@ bool make_q_map(CUtensorMap* map, const void* q, int32_t hq, int64_t total_q, in
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int G>
+template <int G, bool kFp8>
 cudaError_t launch_g(const CUtensorMap& qm, const ExtendTcArgs& a,
                      int64_t grid_z, int32_t max_extend, cudaStream_t s) {
   constexpr int TQ = kRowsPerTile / G;
   const int nqb = (max_extend + kQTiles * TQ - 1) / (kQTiles * TQ);
   static int smem_state[kMaxDevicesHost] = {};
-  cudaError_t e = ensure_smem_limit(extend_tc_kernel<G>, kSmemBytes, smem_state);
+  cudaError_t e = ensure_smem_limit(extend_tc_kernel<G, kFp8>, kSmemBytes, smem_state);
   if (e != cudaSuccess) return e;
   if (grid_z > 65535) return cudaErrorInvalidValue;
   if (nqb > 65535) return cudaErrorInvalidValue;
   dim3 grid(a.hkv, nqb, static_cast<unsigned>(grid_z));
-  extend_tc_kernel<G><<<grid, kThreads, kSmemBytes, s>>>(qm, a);
+  extend_tc_kernel<G, kFp8><<<grid, kThreads, kSmemBytes, s>>>(qm, a);
   return cudaGetLastError();
+}
+
+template <bool kFp8>
+cudaError_t launch_any_g(int G, const CUtensorMap& qm, const ExtendTcArgs& a, int64_t grid_z,
+                         int32_t max_extend, cudaStream_t s) {
+  switch (G) {
+    case 1: return launch_g<1, kFp8>(qm, a, grid_z, max_extend, s);
+    case 2: return launch_g<2, kFp8>(qm, a, grid_z, max_extend, s);
+    case 4: return launch_g<4, kFp8>(qm, a, grid_z, max_extend, s);
+    case 8: return launch_g<8, kFp8>(qm, a, grid_z, max_extend, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_for_pool(const PoolView& pool, int G, const CUtensorMap& qm, const ExtendTcArgs& a,
+                            int64_t grid_z, int32_t max_extend, cudaStream_t s) {
+  return pool.dtype == PKV_DTYPE_FP8_E4M3 ? launch_any_g<true>(G, qm, a, grid_z, max_extend, s)
+                                          : launch_any_g<false>(G, qm, a, grid_z, max_extend, s);
 }
 
 }  // namespace
@@ -748,7 +858,7 @@ cudaError_t launch_extend_tc(const PoolView& pool, const TableView& t, const voi
   a.out = static_cast<__nv_bfloat16*>(out);
   a.hq = num_q_heads;
   a.hkv = pool.num_kv_heads;
-  a.scale_log2 = scale * kLog2e;
+  a.scale_log2 = scale * kLog2e * pool.k_scale;
   a.err = err;
   a.prefix_mode = 0;
   a.nsplit = 1;
@@ -756,13 +866,8 @@ cudaError_t launch_extend_tc(const PoolView& pool, const TableView& t, const voi
   a.nreq = 0;
   a.pre_ml = nullptr;
   a.pre_o = nullptr;
-  switch (G) {
-    case 1: return launch_g<1>(qm, a, batch, max_extend, s);
-    case 2: return launch_g<2>(qm, a, batch, max_extend, s);
-    case 4: return launch_g<4>(qm, a, batch, max_extend, s);
-    case 8: return launch_g<8>(qm, a, batch, max_extend, s);
-  }
-  return cudaErrorInvalidValue;
+  a.v_scale = pool.v_scale;
+  return launch_for_pool(pool, G, qm, a, batch, max_extend, s);
 }
 
 cudaError_t launch_extend_prefix(const PoolView& pool, const TableView& t, const void* q,
@@ -794,7 +899,7 @@ cudaError_t launch_extend_prefix(const PoolView& pool, const TableView& t, const
   a.out = nullptr;
   a.hq = num_q_heads;
   a.hkv = pool.num_kv_heads;
-  a.scale_log2 = scale * kLog2e;
+  a.scale_log2 = scale * kLog2e * pool.k_scale;
   a.err = err;
   a.prefix_mode = 1;
   a.nsplit = nsplit;
@@ -802,14 +907,9 @@ cudaError_t launch_extend_prefix(const PoolView& pool, const TableView& t, const
   a.nreq = batch;
   a.pre_ml = pre_ml;
   a.pre_o = pre_o;
+  a.v_scale = pool.v_scale;
   const int64_t gz = static_cast<int64_t>(num_groups) * nsplit;
-  switch (G) {
-    case 1: return launch_g<1>(qm, a, gz, batch, s);
-    case 2: return launch_g<2>(qm, a, gz, batch, s);
-    case 4: return launch_g<4>(qm, a, gz, batch, s);
-    case 8: return launch_g<8>(qm, a, gz, batch, s);
-  }
-  return cudaErrorInvalidValue;
+  return launch_for_pool(pool, G, qm, a, gz, batch, s);
 }
 
 }  // namespace pkv

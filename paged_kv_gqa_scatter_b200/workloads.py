@@ -733,12 +733,12 @@ def grouped_decode(dtype: str = BF16, groups=((0, 3), (1, 1), (63, 2), (64, 5), 
 # ---------------------------------------------------------------------------
 # FP8 (scaled E4M3) pools.
 # ---------------------------------------------------------------------------
-def with_fp8_pool(wl: DecodeWorkload, k_scale: float = 0.05, v_scale: float = 0.09,
-                  seed: Optional[int] = None) -> DecodeWorkload:
-    """The same decode step over an E4M3 pool: every slot of the touched layers
-    holds random codes (see draw_e4m3_codes); q and the new K/V rows stay the
-    bf16 values of ``wl``; the scales are not powers of two, so the stored
-    codes of the new rows depend on float32 rounding of x * (1 / scale)."""
+def with_fp8_pool(wl, k_scale: float = 0.05, v_scale: float = 0.09, seed: Optional[int] = None):
+    """The same decode step or extend call over an E4M3 pool: every slot of the
+    touched layers holds random codes (see draw_e4m3_codes); q and the new K/V
+    rows stay the bf16 values of ``wl``; the scales are not powers of two, so
+    the stored codes of the new rows depend on float32 rounding of
+    x * (1 / scale)."""
     rng = np.random.Generator(np.random.PCG64(seed_for(8) if seed is None else seed))
     if wl.pool.dtype != BF16 or isinstance(wl.k_planes, TiledPlane):
         raise ValueError("needs a bf16 workload with dict planes")

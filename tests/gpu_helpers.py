@@ -132,7 +132,7 @@ def oracle_decode(wl: W.DecodeWorkload, requests=None, planes=None):
 class DeviceExtend:
     def __init__(self, wl: W.ExtendWorkload, pool: api.KVPool = None, table=None):
         self.wl = wl
-        dt = wl.pool.dtype
+        dt = wl.pool.io_dtype
         self.pool = pool if pool is not None else device_pool(wl.pool, wl.k_planes, wl.v_planes,
                                                               layers=[wl.layer])
         self.table = table if table is not None else api.PageTable(i32(wl.page_table))

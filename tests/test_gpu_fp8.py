@@ -3,6 +3,9 @@
 * store_kv / gather: the stored codes are bit-exact (both sides quantise the
   float32 product x * RN32(1 / scale) with round-to-nearest-even).
 * decode: attention over the dequantised pool, |err| <= 1e-2 + 1e-2 |ref|.
+* extend and cascade decode: attention over the dequantised pool (the
+  tensor cores take f16 operands: E4M3 widens to f16 exactly, bf16 q is
+  converted to f16), same bound as decode.
 * fused norm/RoPE/store: v codes bit-exact (a bf16 value times the inverse
   scale is the same float32 product on both sides); k codes come from an
   fp32 kernel value and a float64 oracle value, so they may differ by one
@@ -160,15 +163,65 @@ def test_fp8_rope_store():
     assert np.array_equal(_codes(pool.v[0])[others], vp0[0][others])
 
 
-def test_fp8_unsupported_calls():
-    wl = W.with_fp8_pool(W.decode_small())
+def _oracle_extend(wl, rows=None):
+    kp = {l: a.copy() for l, a in wl.k_planes.items()}
+    vp = {l: a.copy() for l, a in wl.v_planes.items()}
+    oracle.store_kv_fp8(kp, vp, wl.layer, wl.k_new, wl.v_new, wl.out_loc, wl.pool.num_kv_heads, D,
+                        wl.pool.k_scale, wl.pool.v_scale)
+    return oracle.extend_attn(wl.q, oracle.dequant_planes(kp, wl.pool.k_scale, [wl.layer]),
+                              oracle.dequant_planes(vp, wl.pool.v_scale, [wl.layer]), wl.layer,
+                              wl.page_table, wl.table_idx, wl.prefix_lens, wl.extend_lens,
+                              wl.q_offsets, wl.pool.page_size, wl.scale, rows=rows)
+
+
+@pytest.mark.parametrize("hq,hkv,page_size", [(16, 8, 1), (32, 8, 1), (8, 8, 1), (64, 8, 1), (16, 8, 64)])
+def test_fp8_extend_matches_oracle(hq, hkv, page_size):
+    """Extend over an E4M3 pool: ragged prefixes 0 / 37 / 130 with chunks of
+    45 / 1 / 200 tokens; the chunk's own rows are quantised by store_kv."""
+    wl = W.with_fp8_pool(W.extend_small(num_q_heads=hq, num_kv_heads=hkv, page_size=page_size), seed=hq)
+    from gpu_helpers import DeviceExtend
+    d = DeviceExtend(wl)
+    d.run()
+    torch.cuda.synchronize()
+    assert int(d.err.item()) == 0
+    tol_check(from_dev(d.out), _oracle_extend(wl), W.BF16, f"fp8 extend hq={hq} P={page_size}")
+
+
+def test_fp8_extend_chunked_prefill_sampled():
+    """The 2048-token chunk at prefix 6144 (Hq 32, Hkv 8) over an E4M3 pool;
+    64 sampled rows against the oracle."""
+    wl = W.with_fp8_pool(W.chunked_prefill_step(step=3).extend)
+    from gpu_helpers import DeviceExtend
+    d = DeviceExtend(wl)
+    d.run()
+    torch.cuda.synchronize()
+    assert int(d.err.item()) == 0
+    rows = np.sort(np.random.default_rng(4).choice(wl.total_q, 64, replace=False))
+    exp = _oracle_extend(wl, rows=rows)
+    tol_check(from_dev(d.out)[rows], exp[rows], W.BF16, "fp8 extend chunk c3")
+
+
+def test_fp8_cascade_decode():
+    gd = W.grouped_decode(groups=((64, 3), (1000, 20), (0, 2)), max_suffix=150, seed=71)
+    wl = W.with_fp8_pool(gd.decode, seed=72)
     d = DeviceDecode(wl)
+    api.store_kv(d.pool, 0, d.k_new, d.v_new, d.out_loc, d.err)
+    mp = int(gd.group_prefix_lens.max())
+    ws = api.decode_cascade_workspace(wl.batch, wl.num_q_heads, mp)
     out = torch.empty_like(d.q)
-    qo = torch.tensor([0, 1], dtype=torch.int32, device="cuda")
+    api.decode_attn_cascade(d.pool, 0, d.q, d.table, d.table_idx, d.seq_lens, i32(gd.group_offsets),
+                            i32(gd.group_prefix_lens), mp, out, ws, scale=wl.scale, dev_err=d.err)
+    torch.cuda.synchronize()
+    assert int(d.err.item()) == 0
+    kp, vp = _oracle_store(wl)
+    tol_check(from_dev(out), _oracle_decode(wl, kp, vp), W.BF16, "fp8 cascade decode")
+
+
+def test_fp32_cascade_unsupported():
+    gd = W.grouped_decode(W.F32, groups=((64, 2),), seed=73)
+    d = DeviceDecode(gd.decode)
+    ws = api.decode_cascade_workspace(gd.decode.batch, gd.decode.num_q_heads, 64)
     with pytest.raises(RuntimeError, match="unsupported"):
-        api.extend_attn(d.pool, 0, d.q[:1], d.table, d.table_idx[:1], i32([0]), i32([1]), qo, 1,
-                        out[:1], scale=wl.scale)
-    ws = api.decode_cascade_workspace(wl.batch, wl.num_q_heads, 16)
-    with pytest.raises(RuntimeError, match="unsupported"):
-        api.decode_attn_cascade(d.pool, 0, d.q, d.table, d.table_idx, d.seq_lens, i32([0, wl.batch]),
-                                i32([16]), 16, out, ws, scale=wl.scale)
+        api.decode_attn_cascade(d.pool, 0, d.q, d.table, d.table_idx, d.seq_lens, i32(gd.group_offsets),
+                                i32(gd.group_prefix_lens), 64, torch.empty_like(d.q), ws,
+                                scale=gd.decode.scale)
