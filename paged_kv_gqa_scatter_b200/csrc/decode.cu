@@ -29,6 +29,12 @@
 //  * A piece that covers a whole request writes the final output; other
 //    pieces write an un-normalised fp32 partial plus (max, sum) to the
 //    workspace and decode_combine_kernel merges them.
+//  * Cascade suffix pass (cascade.cu): each request starts at its own table
+//    column, every piece writes a partial, and the combine kernel also merges
+//    the shared-prefix partials.
+//  * FP8 (E4M3) pools: 32 tokens per stage (1 KB rows); codes widen exactly to
+//    half and then float; the K scale is folded into the softmax scale and
+//    the V scale into the output.
 #include <cuda_bf16.h>
 
 #include "common.cuh"
