@@ -21,8 +21,9 @@
  * --------------------------------
  * Ownership: the caller owns every buffer passed in (device memory unless a
  *   parameter says "host").  No call keeps a pointer after it returns, and no
- *   call allocates device memory; scratch space comes from a caller-provided
- *   workspace whose size a *_workspace_bytes query returns.
+ *   compute call allocates device memory; scratch space comes from a
+ *   caller-provided workspace whose size a *_workspace_bytes query returns,
+ *   or from a pkv_workspace object (the only calls that allocate).
  * Streams: every compute call is asynchronous on the given stream (0 = the
  *   legacy default stream) and never synchronises the host.
  * Errors: calls return a pkv_status.  Host-side checks (null pointers,
@@ -198,6 +199,38 @@ int pkv_qk_norm_rope_store(const pkv_pool* pool, int32_t layer, const void* qkv,
                            const void* k_norm_weight, float eps, const void* out_loc,
                            int32_t out_loc_is_i64, int64_t n_tokens, void* q_out,
                            int32_t* dev_err, pkv_stream_t stream);
+
+/*
+ * Workspace objects -- the one part of the library that allocates.  A caller
+ * that does not want to size and own scratch memory creates one per stream
+ * at start-up (before any CUDA-graph capture) on the current device:
+ *
+ *   pkv_workspace_create(max_batch, max_q_heads, max_prefix_len, &ws)
+ *     allocates (cudaMalloc) a buffer large enough for pkv_decode_attn and
+ *     pkv_decode_attn_cascade at up to max_batch requests of max_q_heads
+ *     heads (cascade prefixes up to max_prefix_len; 0 if unused; extend
+ *     needs no workspace) and a zeroed int32 device error word.
+ *     PKV_ERR_CUDA if an allocation fails; *ws is NULL then.
+ *   pkv_workspace_buffer(ws, &bytes) -> the buffer and its size, to pass as
+ *     `workspace` / `workspace_bytes`.
+ *   pkv_workspace_error_word(ws) -> the device error word, to pass as
+ *     `dev_err`.
+ *   pkv_read_device_error(ws, stream, &code) -> waits for the stream, stores
+ *     the accumulated pkv_device_error bits in *code and clears the word.
+ *   pkv_workspace_destroy(ws) frees both allocations (NULL is a no-op); no
+ *     call that uses them may still be pending.
+ *
+ * The pages have no counterpart; their backends allocate such buffers once
+ * when the engine starts.  A workspace must not be shared by calls that may
+ * overlap on the GPU.
+ */
+typedef struct pkv_workspace pkv_workspace;
+int pkv_workspace_create(int32_t max_batch, int32_t max_q_heads, int64_t max_prefix_len,
+                         pkv_workspace** ws);
+void pkv_workspace_destroy(pkv_workspace* ws);
+void* pkv_workspace_buffer(const pkv_workspace* ws, size_t* bytes);
+int32_t* pkv_workspace_error_word(const pkv_workspace* ws);
+int pkv_read_device_error(pkv_workspace* ws, pkv_stream_t stream, int32_t* code);
 
 /*
  * selftest_wait_timeout -- exercises the bounded wait of the pipelined

@@ -41,6 +41,11 @@ SIGNATURES = {
                                               c_i32, c_vp, c_i64, c_vp, c_vp, ctypes.c_float, c_vp,
                                               c_i32, c_i64, c_vp, c_vp, c_vp]),
     "pkv_selftest_wait_timeout": (ctypes.c_int, [c_vp, c_vp]),
+    "pkv_workspace_create": (ctypes.c_int, [c_i32, c_i32, c_i64, ctypes.POINTER(c_vp)]),
+    "pkv_workspace_destroy": (None, [c_vp]),
+    "pkv_workspace_buffer": (c_vp, [c_vp, ctypes.POINTER(c_size)]),
+    "pkv_workspace_error_word": (c_vp, [c_vp]),
+    "pkv_read_device_error": (ctypes.c_int, [c_vp, c_vp, ctypes.POINTER(c_i32)]),
     "pkv_gather_kv": (ctypes.c_int, [ctypes.POINTER(PkvPool), c_i32, ctypes.POINTER(PkvPageTable),
                                      c_vp, c_vp, c_vp, c_i32, c_vp, c_vp, c_vp, c_vp]),
     "pkv_decode_workspace_bytes": (c_size, [c_i32, c_i32]),

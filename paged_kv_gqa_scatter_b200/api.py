@@ -33,13 +33,63 @@ def _stream_ptr(stream: Optional[torch.cuda.Stream]) -> int:
     return int(s.cuda_stream)
 
 
-def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
-    return None if t is None else int(t.data_ptr())
+class Workspace:
+    """A library-owned workspace (pkv_workspace_create): a scratch buffer for
+    decode / cascade decode and a device error word.  Pass it as `workspace`
+    and as `dev_err`; read_device_error() waits for the stream and returns and
+    clears the error bits."""
+
+    def __init__(self, max_batch: int, max_q_heads: int, max_prefix_len: int = 0):
+        lib = _lib.load()
+        h = ctypes.c_void_p()
+        _lib.check(lib.pkv_workspace_create(max_batch, max_q_heads, max_prefix_len, ctypes.byref(h)),
+                   "workspace_create")
+        self._h = h
+
+    def buffer(self):
+        n = ctypes.c_size_t()
+        p = _lib.load().pkv_workspace_buffer(self._h, ctypes.byref(n))
+        return int(p), int(n.value)
+
+    def error_word(self) -> int:
+        return int(_lib.load().pkv_workspace_error_word(self._h))
+
+    def read_device_error(self, stream=None) -> int:
+        code = ctypes.c_int32()
+        _lib.check(_lib.load().pkv_read_device_error(self._h, _stream_ptr(stream), ctypes.byref(code)),
+                   "read_device_error")
+        return int(code.value)
+
+    def close(self) -> None:
+        if self._h is not None and self._h.value:
+            _lib.load().pkv_workspace_destroy(self._h)
+        self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def _ptr(t) -> Optional[int]:
+    if t is None:
+        return None
+    if isinstance(t, Workspace):
+        return t.error_word()
+    return int(t.data_ptr())
+
+
+def _ws(w):
+    """(pointer, bytes) of a workspace tensor or Workspace object."""
+    if isinstance(w, Workspace):
+        return w.buffer()
+    return int(w.data_ptr()), w.numel() * w.element_size()
 
 
 def _require_cuda(*ts):
     for t in ts:
-        if t is not None and not t.is_cuda:
+        if t is not None and not isinstance(t, Workspace) and not t.is_cuda:
             raise ValueError("pkv calls take CUDA tensors")
 
 
@@ -188,8 +238,7 @@ def decode_attn(pool: KVPool, layer: int, q: torch.Tensor, table: PageTable,
     lib = _lib.load()
     _lib.check(lib.pkv_decode_attn(ctypes.byref(pool.c), layer, q.data_ptr(), Hq,
                                    ctypes.byref(table.c), table_idx.data_ptr(), seq_lens.data_ptr(),
-                                   B, scale, out.data_ptr(), workspace.data_ptr(),
-                                   workspace.numel() * workspace.element_size(), _ptr(dev_err),
+                                   B, scale, out.data_ptr(), *_ws(workspace), _ptr(dev_err),
                                    _stream_ptr(stream)), "decode_attn")
 
 
@@ -248,8 +297,8 @@ def decode_attn_cascade(pool: KVPool, layer: int, q: torch.Tensor, table: PageTa
     _lib.check(lib.pkv_decode_attn_cascade(
         ctypes.byref(pool.c), layer, q.data_ptr(), Hq, ctypes.byref(table.c), table_idx.data_ptr(),
         seq_lens.data_ptr(), B, group_offsets.data_ptr(), group_prefix_lens.data_ptr(),
-        group_prefix_lens.numel(), int(max_prefix_len), scale, out.data_ptr(), workspace.data_ptr(),
-        workspace.numel() * workspace.element_size(), _ptr(dev_err), _stream_ptr(stream)),
+        group_prefix_lens.numel(), int(max_prefix_len), scale, out.data_ptr(), *_ws(workspace),
+        _ptr(dev_err), _stream_ptr(stream)),
         "decode_attn_cascade")
 
 
