@@ -11,7 +11,8 @@
  *   [P5] "Mini-SGLang 完整剖析" (blog.rzhang-lab.cn/post/3)
  *        §1.2 prefill vs decode, §1.3 KV cache, §1.4 paged pool and prefix
  *        sharing, §4.2.3 request length fields, §4.4.3 pool tensor,
- *        §4.6.4 page-table metadata, §4.6.7 attention layer / store_kv,
+ *        §4.5.6 shared RotaryEmbedding, §4.6.4 page-table metadata,
+ *        §4.6.6 CUDA-graph capture, §4.6.7 attention layer / store_kv,
  *        §4.9.4 store kernel shape checks.
  *   [P4] "深入解析 mini-sglang" (yunpan.plus), chunked prefill.
  *   [P3] "mini-sglang 深度分析报告" (nightvoyager.top), design notes
@@ -37,9 +38,13 @@
  *   each internal wait gives up after about one second and sets
  *   PKV_DEV_ERR_TIMEOUT.
  * Element types: bf16 (the product path), fp32 (a check build of the same
- *   kernels for tighter numerical comparison) and a scaled FP8 E4M3 pool
- *   (store, gather, fused store and decode; see pkv_pool).  head_dim must
- *   be 128.
+ *   kernels for tighter numerical comparison; no cascade decode) and a
+ *   scaled FP8 E4M3 pool (every call; see pkv_pool).  head_dim must be 128.
+ * Launch overlap: the store calls let the next kernel launch early
+ *   (programmatic dependent launch); decode waits for the preceding kernel
+ *   before it reads any input, so inputs written by that kernel are safe.
+ * CUDA graphs: every compute call can be captured; make the first call on
+ *   a device outside capture (it sets kernel attributes once).
  */
 #ifndef PKV_H_
 #define PKV_H_
