@@ -110,3 +110,61 @@ def test_workspace_size_grows_with_batch_and_heads():
     c = lib.pkv_decode_workspace_bytes(64, 32)
     assert 0 < a < b and a < c
     assert lib.pkv_decode_workspace_bytes(-1, 16) == 0
+
+
+def test_host_validation_of_the_newer_calls():
+    lib = _lib.load()
+    dummy = 4096
+    P = ctypes.byref
+    t = _lib.PkvPageTable(entries=dummy, rows=4, cols=64, row_stride=64)
+    row = (16 + 2 * 8) * 128
+    # qk_norm_rope_store: (pool, layer, qkv, stride, hq, pos, pos64, cache, maxpos, qw, kw, eps,
+    #                      loc, loc64, n, q_out, err, stream)
+    rope = lambda **kw: lib.pkv_qk_norm_rope_store(
+        P(kw.get("pool", _pool())), 0, kw.get("qkv", dummy), kw.get("stride", row), 16, dummy, 0, dummy,
+        kw.get("maxpos", 4096), None, None, kw.get("eps", 1e-6), dummy, 0, kw.get("n", 4), dummy, None, None)
+    assert rope(qkv=None) == 1
+    assert rope(eps=-1.0) == 1
+    assert rope(maxpos=0) == 1
+    assert rope(stride=row - 8) == 1
+    assert rope(qkv=dummy + 2) == 3
+    assert rope(n=0) == 0
+    # cascade decode: (pool, layer, q, hq, table, ti, sl, batch, off, pre, groups, maxp, scale, out,
+    #                  ws, ws_bytes, err, stream)
+    cas = lambda **kw: lib.pkv_decode_attn_cascade(
+        P(kw.get("pool", _pool())), 0, dummy, 16, P(t), dummy, dummy, kw.get("batch", 4), dummy, dummy,
+        kw.get("groups", 1), kw.get("maxp", 32), 0.1, dummy, dummy, kw.get("ws", 1 << 30), None, None)
+    assert cas(pool=_pool(dtype=1, slot_stride=1024, layer_stride=64 * 1024)) == 2  # fp32 pool
+    assert cas(groups=0) == 1
+    assert cas(groups=5) == 1          # more groups than requests
+    assert cas(maxp=65) == 6           # prefix longer than the table
+    assert cas(ws=16) == 4
+    assert cas(batch=0) == 0
+    # FP8 pools need finite positive scales; rows written into them are bf16.
+    f8 = lambda ks, vs: _pool(dtype=2, slot_stride=1024, layer_stride=64 * 1024, k_scale=ks, v_scale=vs)
+    for ks, vs in ((0.0, 1.0), (1.0, -2.0), (float("inf"), 1.0), (float("nan"), 1.0)):
+        assert lib.pkv_store_kv(P(f8(ks, vs)), 0, dummy, 1024, dummy, 1024, dummy, 0, 1, None, None) == 1
+    assert lib.pkv_store_kv(P(f8(0.05, 0.09)), 0, dummy, 1024, dummy, 1024, dummy, 0, 0, None, None) == 0
+    # bf16 rows of 1024 elements: a stride of 1028 bf16 elements breaks 16-byte rows
+    assert lib.pkv_store_kv(P(f8(0.05, 0.09)), 0, dummy, 1028, dummy, 1024, dummy, 0, 1, None, None) == 3
+    # self-test and workspace objects
+    assert lib.pkv_selftest_wait_timeout(None, None) == 1
+    h = ctypes.c_void_p()
+    assert lib.pkv_workspace_create(0, 16, 0, P(h)) == 1 and not h.value
+    assert lib.pkv_workspace_create(4, 16, -1, P(h)) == 1
+    assert lib.pkv_workspace_create(4, 16, 0, None) == 1
+    code = ctypes.c_int32()
+    assert lib.pkv_read_device_error(None, None, P(code)) == 1
+    n = ctypes.c_size_t(7)
+    assert lib.pkv_workspace_buffer(None, P(n)) is None and n.value == 0
+    assert lib.pkv_workspace_error_word(None) is None
+    lib.pkv_workspace_destroy(None)  # a no-op
+
+
+def test_cascade_workspace_size():
+    lib = _lib.load()
+    a = lib.pkv_decode_cascade_workspace_bytes(64, 16, 0)
+    b = lib.pkv_decode_cascade_workspace_bytes(64, 16, 4096)
+    c = lib.pkv_decode_cascade_workspace_bytes(64, 16, 32768)
+    assert lib.pkv_decode_workspace_bytes(64, 16) <= a < b < c
+    assert lib.pkv_decode_cascade_workspace_bytes(64, 16, -1) == 0
