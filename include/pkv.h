@@ -318,9 +318,12 @@ int pkv_decode_attn(const pkv_pool* pool, int32_t layer, const void* q, int32_t 
  * Limits and behaviour:
  *  - Returns PKV_ERR_TOO_LARGE, launching nothing, when
  *    pkv_decode_workspace_bytes(batch, num_q_heads) exceeds that size.
- *  - The first call on each device (with it current) looks up the array's
- *    device address and caches it; make that first call outside any stream
- *    capture.
+ *  - Every call made outside stream capture (with its device current) looks
+ *    up the array's device address and caches it per device; a call made
+ *    while its stream is captured reuses the cached address.  Make the first
+ *    call on a device outside any stream capture, and, after a device reset
+ *    (which reloads the library's device code and may move the array), make
+ *    one more uncaptured call before capturing again.
  *  - All calls on a device share the array: calls that can overlap on the GPU
  *    (unordered streams) race; calls ordered on one stream are safe.  Nothing
  *    in the array needs to start at zero.

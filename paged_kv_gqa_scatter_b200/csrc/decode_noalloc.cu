@@ -11,10 +11,14 @@
 // Properties a caller must know:
 //  * The array is kNoAllocScratchBytes (16 MiB) on every device that loads the
 //    library, held until the process exits.
-//  * Host code cannot use the array's name as a device address.  The first
-//    call on each device (with that device current) looks the address up with
-//    cudaGetSymbolAddress and caches it; make that first call outside any
-//    stream capture.
+//  * Host code cannot use the array's name as a device address.  Every call
+//    made outside stream capture (with its device current) looks the address
+//    up with cudaGetSymbolAddress and caches it per device, so a device reset
+//    that reloads the library's device code is picked up by the next such
+//    call.  A call made while its stream is being captured uses the cached
+//    address (or looks it up if there is none yet); make the first call on a
+//    device outside any stream capture, and make another one after a device
+//    reset before capturing again.
 //  * Every call on a device shares the one array, so calls that may overlap on
 //    the GPU (different streams without ordering between them) race and can
 //    corrupt each other's results.  Calls ordered on one stream are safe.
@@ -37,12 +41,16 @@ static __device__ __align__(256) unsigned char g_decode_scratch[kNoAllocScratchB
 std::mutex g_setup_mu;
 void* g_scratch_ptr[kMaxDevices] = {};
 
-// Device address of g_decode_scratch on the current device (looked up once).
-int scratch_address(void** out) {
+// Device address of g_decode_scratch on the current device.  Looked up again
+// on every call that is not being captured; a call under capture reuses the
+// address cached by the last uncaptured call.
+int scratch_address(cudaStream_t stream, void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return PKV_ERR_CUDA;
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(stream, &cs) != cudaSuccess) return PKV_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_setup_mu);
-  if (g_scratch_ptr[dev] == nullptr) {
+  if (cs == cudaStreamCaptureStatusNone || g_scratch_ptr[dev] == nullptr) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || p == nullptr) return PKV_ERR_CUDA;
     g_scratch_ptr[dev] = p;
@@ -64,7 +72,7 @@ int pkv_decode_attn_noalloc(const pkv_pool* pool, int32_t layer, const void* q, 
   if (batch < 0 || num_q_heads < 1) return PKV_ERR_INVALID_ARG;
   if (pkv_decode_workspace_bytes(batch, num_q_heads) > kNoAllocScratchBytes) return PKV_ERR_TOO_LARGE;
   void* scratch = nullptr;
-  const int st = scratch_address(&scratch);
+  const int st = scratch_address(static_cast<cudaStream_t>(stream), &scratch);
   if (st != PKV_OK) return st;
   return pkv_decode_attn(pool, layer, q, num_q_heads, table, table_idx, seq_lens, batch, scale, out,
                          scratch, kNoAllocScratchBytes, dev_err, stream);

@@ -309,7 +309,13 @@ def decode_qwen3_06b(dtype: str = BF16, batch: int = 64, min_len: int = 512, max
 # ---------------------------------------------------------------------------
 # Workload 3: Qwen3-8B-shaped large decode batch over a 36-layer pool.
 # ---------------------------------------------------------------------------
-def decode_qwen3_8b(num_pages: int, dtype: str = BF16, batch: int = 256, min_len: int = 1024,
+# Physical 16-token pages of the Qwen3-8B decode pool: 36 layers x 45,056
+# pages x 16 slots x 4 KB = 106 GB, about 0.55 of a B200's memory.  Fixed (not
+# sized from free memory) so that every run builds the same page aliasing.
+QWEN3_8B_POOL_PAGES = 45_056
+
+
+def decode_qwen3_8b(num_pages: int = QWEN3_8B_POOL_PAGES, dtype: str = BF16, batch: int = 256, min_len: int = 1024,
                     max_len: int = 32768, num_layers: int = 36, page_size: int = 16,
                     num_q_heads: int = 32, num_kv_heads: int = 8, block_slots: int = 1 << 16,
                     seed: Optional[int] = None) -> DecodeWorkload:

@@ -222,18 +222,27 @@ def test_decode_qwen3_06b_full():
 
 
 def test_decode_qwen3_8b_sampled():
-    """Batch 256, log-uniform 1k-32k, page_size 16, aliased pages; last layer of 36;
-    16 sampled requests (longest and shortest included) compared."""
-    wl = W.decode_qwen3_8b(num_pages=20000)
-    wl.layer = 35
-    d = DeviceDecode(wl, pool=device_pool(wl.pool, wl.k_planes, wl.v_planes, layers=[35]))
-    d.run()
+    """Batch 256, log-uniform 1k-32k, page_size 16, on the pool the benchmark
+    builds (36 layers of W.QWEN3_8B_POOL_PAGES pages, so the same aliased
+    pages); layers 0 and 35; 16 sampled requests (longest and shortest
+    included) compared on each."""
+    wl = W.decode_qwen3_8b()
+    assert wl.pool.num_slots == W.QWEN3_8B_POOL_PAGES * 16 and wl.pool.num_layers == 36
+    pool = device_pool(wl.pool, wl.k_planes, wl.v_planes, layers=[0, 35])
     lens = wl.seq_lens
     req = sorted(set([int(np.argmax(lens)), int(np.argmin(lens))] +
                      np.random.default_rng(3).choice(wl.batch, 14, replace=False).tolist()))
-    exp, _ = oracle_decode(wl, requests=req)
-    tol_check(from_dev(d.out)[req], exp[req], W.BF16, "decode-qwen3-8b")
-    assert _err(d.err) == 0
+    table = None
+    for layer in (0, 35):
+        wl.layer = layer
+        d = DeviceDecode(wl, pool=pool, table=table)
+        table = d.table
+        d.run()
+        exp, _ = oracle_decode(wl, requests=req)
+        tol_check(from_dev(d.out)[req], exp[req], W.BF16, f"decode-qwen3-8b layer {layer}")
+        assert _err(d.err) == 0
+    del pool
+    torch.cuda.empty_cache()
 
 
 # ---------------------------------------------------------------------------
@@ -269,34 +278,55 @@ def test_extend_zero_length_requests_in_batch():
     tol_check(from_dev(d.out), exp, W.BF16, "extend with empty chunks")
 
 
-def test_extend_chunked_prefill_step():
-    """One 2048-token chunk at prefix 6144 (step 3 of 8192-token prompts): 96 sampled
-    query rows, including the first and the last rows of the chunk."""
-    mix = W.chunked_prefill_step(step=3)
+def _chunk_rows(prefix: int, e: int, hq: int, hkv: int, seed: int):
+    """Rows to compare in a chunk: the first and last token of every 128-row
+    query tile (128 / G tokens), the tokens whose visible keys end on a
+    64-key step boundary or just past one (the diagonal steps), and seeded
+    others."""
+    tq = 128 // (hq // hkv)
+    rows = set()
+    for t0 in range(0, e, tq):
+        rows.update([t0, min(e, t0 + tq) - 1])
+    for i in range(e):
+        if (prefix + i + 1) % 64 in (0, 1):
+            rows.add(i)
+    rows.update(np.random.default_rng(seed).choice(e, 32, replace=False).tolist())
+    return sorted(rows)
+
+
+@pytest.mark.parametrize("step", [0, 1, 2, 3])
+def test_extend_chunked_prefill_step(step):
+    """Chunk `step` (prefix 2048 * step) of an 8192-token prompt in 2048-token
+    chunks, at full size: the rows of _chunk_rows compared; then the step's
+    128-request decode batch on the same pool, every output compared."""
+    mix = W.chunked_prefill_step(step=step)
     wl = mix.extend
     d = DeviceExtend(wl)
     d.run()
-    rows = sorted(set([0, 1, 2, 63, 64, 127, 128, 2047, 2046] +
-                      np.random.default_rng(9).choice(2048, 87, replace=False).tolist()))
+    rows = _chunk_rows(int(wl.prefix_lens[0]), int(wl.extend_lens[0]), wl.num_q_heads,
+                       wl.pool.num_kv_heads, 9 + step)
     exp, planes = oracle_extend(wl, rows=rows)
-    tol_check(from_dev(d.out)[rows], exp[rows], W.BF16, "chunked prefill extend")
-    # The same step's decode batch runs on the same pool after the extend.
+    tol_check(from_dev(d.out)[rows], exp[rows], W.BF16, f"chunked prefill extend c{step}")
     dd = DeviceDecode(mix.decode, pool=d.pool, table=d.table)
     dd.run()
     expd, _ = oracle_decode(mix.decode, planes=planes)
-    tol_check(from_dev(dd.out), expd, W.BF16, "chunked prefill decode")
+    tol_check(from_dev(dd.out), expd, W.BF16, f"chunked prefill decode c{step}")
     assert _err(d.err) == 0 and _err(dd.err) == 0
 
 
 def test_radix_shared_prefix_extend_then_decode():
     """Shared 4096-token prefix, 256 suffixes extended in one call, then 64 decode steps;
-    sampled requests checked after the extend and after decode steps 1 and 64."""
+    34 sampled requests (the shortest and longest suffixes included) checked
+    after the extend and after decode steps 1 and 64."""
     rs = W.radix_shared_prefix()
     wl = rs.extend
     d = DeviceExtend(wl)
     d.run()
     rng = np.random.default_rng(11)
-    req = sorted(rng.choice(wl.batch, 8, replace=False).tolist())
+    el = wl.extend_lens
+    req = sorted(set([int(np.argmin(el)), int(np.argmax(el))] +
+                     rng.choice(wl.batch, 32, replace=False).tolist()))
+    assert len(req) >= 32
     rows = np.concatenate([np.arange(wl.q_offsets[r], wl.q_offsets[r + 1]) for r in req])
     exp, planes = oracle_extend(wl, rows=rows)
     tol_check(from_dev(d.out)[rows], exp[rows], W.BF16, "radix extend")
