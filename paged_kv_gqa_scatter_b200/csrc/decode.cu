@@ -119,17 +119,19 @@ __host__ __device__ inline DecodeSmem decode_smem_layout(int batch, int hkv, int
   return L;
 }
 
-// Transposing butterfly over the 16 lanes of a half-warp.  On entry every lane
-// holds V partial sums v[0..V); on exit lane c holds the complete sums of
-// values (V/16)*c .. (V/16)*c + V/16 - 1 (V >= 16), or of value c >> (4 - log2 V)
-// (V < 16, lanes sharing a value hold the same sum).
-template <int V>
-__device__ __forceinline__ void transpose_reduce16(float (&v)[V], int c) {
+// Transposing butterfly over groups of D consecutive lanes (D = 8 or 16).  On
+// entry every lane holds V partial sums v[0..V); on exit lane d (its index in
+// the group) holds the complete sums of values (V/D)*d .. (V/D)*d + V/D - 1
+// (V >= D), or of value d >> (log2 D - log2 V) (V < D; lanes sharing a value
+// hold the same sum).  Each level halves the values a lane keeps, so the
+// reduction costs about one shuffle per complete sum instead of log2 D.
+template <int V, int D>
+__device__ __forceinline__ void transpose_reduce(float (&v)[V], int d) {
   int n = V;
 #pragma unroll
-  for (int off = 8; off >= 1; off >>= 1) {
+  for (int off = D / 2; off >= 1; off >>= 1) {
     if (n >= 2) {
-      const bool upper = (c & off) != 0;
+      const bool upper = (d & off) != 0;
 #pragma unroll
       for (int k = 0; k < V / 2; ++k) {
         if (k < n / 2) {
@@ -145,17 +147,52 @@ __device__ __forceinline__ void transpose_reduce16(float (&v)[V], int c) {
   }
 }
 
+constexpr int ilog2c(int x) { return x <= 1 ? 0 : 1 + ilog2c(x / 2); }
+
+// p values of query heads 0..G-1 for one token, from the warp's p buffer.
+template <int G>
+__device__ __forceinline__ void load_p(const float* src, float (&p)[G]) {
+  if constexpr (G == 1) {
+    p[0] = src[0];
+  } else if constexpr (G == 2) {
+    const float2 x = *reinterpret_cast<const float2*>(src);
+    p[0] = x.x;
+    p[1] = x.y;
+  } else {
+#pragma unroll
+    for (int k = 0; k < G; k += 4) {
+      const float4 x = *reinterpret_cast<const float4*>(src + k);
+      p[k] = x.x;
+      p[k + 1] = x.y;
+      p[k + 2] = x.z;
+      p[k + 3] = x.w;
+    }
+  }
+}
+
 template <typename E, int G>
 __global__ void __launch_bounds__(32 * 9, 1) decode_split_kernel(const DecodeArgs a) {
   constexpr int T = DecodeTraits<E>::kTokensPerStage;
   constexpr int SUB = (64 / G < T) ? 64 / G : T;  // tokens per softmax sub-step
-  constexpr int HALF = SUB / 2;                    // tokens per lane per sub-step
-  constexpr int V = HALF * G;                      // partial sums per lane
-  constexpr int NV = V >= 16 ? V / 16 : 1;         // complete sums per lane after reduce
-  constexpr int LPH = 16 / G;                      // lanes per head within a half
+  constexpr int HALF = SUB / 2;                    // PV: tokens per lane per sub-step
+  // Scores: D lanes share a token (each owns 16/D units of 8 dims: units d
+  // and d + D), TL = 32/D tokens are in flight per warp step, and a lane
+  // keeps V = SPL*G partial sums per sub-step.  D = 8 halves the reduction
+  // of D = 16; wide groups (G = 8, whose q would not fit in registers) and
+  // FP8 rows (8-byte units, where D = 8 would put two rows on one bank
+  // range) keep D = 16.
+  constexpr int D = (G >= 8 || sizeof(E) == 1) ? 16 : 8;
+  constexpr int TL = 32 / D;
+  constexpr int UPL = 16 / D;                      // 8-element units per lane
+  constexpr int SPL = SUB / TL;                    // tokens per lane per sub-step
+  constexpr int V = SPL * G;                       // partial sums per lane
+  constexpr int NV = V >= D ? V / D : 1;           // complete sums per lane after reduce
+  constexpr int LPH = D / G;                       // lanes of a token group holding one head
+  constexpr int kLog2D = ilog2c(D);
+  constexpr int kLog2V = ilog2c(V);
   constexpr int ESZ = sizeof(E);
   using IO = typename DecodeTraits<E>::IO;
-  constexpr int kLog2V = V >= 16 ? 4 : (V == 8 ? 3 : (V == 4 ? 2 : (V == 2 ? 1 : 0)));
+  static_assert(SUB % TL == 0 && NV <= SPL, "decode sub-step shape");
 
   extern __shared__ __align__(128) uint8_t smem[];
   // Let the combine kernel be scheduled early; it waits for this grid anyway.
@@ -373,9 +410,22 @@ __global__ void __launch_bounds__(32 * 9, 1) decode_split_kernel(const DecodeArg
   }
 
   // ============================= consumers ==================================
+  // Scores use the token-group lane map (tl, d) = (lane / D, lane % D); the
+  // PV product uses (half, c) = (lane / 16, lane % 16): lane c owns dims
+  // 8c .. 8c+7 and half picks even or odd tokens.  The p values pass from the
+  // first map to the second through the warp's p buffer [SUB][G].
   const int g = warp - 1;  // KV head
   if (g >= ncons) return;
   const int c = lane & 15, half = lane >> 4;
+  const int tl = lane / D, d = lane % D;
+  // Head and value index of the complete scores this lane holds after the
+  // reduction; for V < D, lanes sharing a value let only the first add it
+  // to the running sum.
+  const int idx0 = V >= D ? NV * d : (d >> (kLog2D - kLog2V));
+  const int hl = idx0 / SPL;
+  const bool owner = V >= D || (d & ((D >> kLog2V) - 1)) == 0;
+  // A lane holding scores of head hh (used to broadcast per-head values).
+  auto head_lane = [](int hh) { return hh * LPH; };
   float* pw = psm + g * SUB * G;  // this warp's p buffer [SUB][G]
   const IO* qbase = static_cast<const IO*>(a.q);
   IO* obase = static_cast<IO*>(a.out);
@@ -390,25 +440,27 @@ __global__ void __launch_bounds__(32 * 9, 1) decode_split_kernel(const DecodeArg
       asm volatile("prefetch.global.L2 [%0];" ::"l"(qbase + ((int64_t)(r + 1) * a.hq + g * G) * kHeadDim +
                                                       lane * (128 / static_cast<int>(sizeof(IO)))));
 
-    float2 q2[G][4];
+    // q of this lane's units (pre-scaled by scale * log2 e).
+    float2 q2[G][UPL][4];
 #pragma unroll
     for (int hh = 0; hh < G; ++hh) {
-      load8<IO>(qbase + ((int64_t)r * a.hq + g * G + hh) * kHeadDim + 8 * c, q2[hh]);
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        q2[hh][e].x *= a.scale_log2;
-        q2[hh][e].y *= a.scale_log2;
+      for (int m = 0; m < UPL; ++m) {
+        load8<IO>(qbase + ((int64_t)r * a.hq + g * G + hh) * kHeadDim + 8 * (d + D * m), q2[hh][m]);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          q2[hh][m][e].x *= a.scale_log2;
+          q2[hh][m][e].y *= a.scale_log2;
+        }
       }
     }
     float2 o2[G][4];
-    float lsum[G];
 #pragma unroll
-    for (int hh = 0; hh < G; ++hh) {
-      lsum[hh] = 0.f;
+    for (int hh = 0; hh < G; ++hh)
 #pragma unroll
       for (int e = 0; e < 4; ++e) o2[hh][e] = make_float2(0.f, 0.f);
-    }
-    float m_run = -INFINITY;  // running max of this lane's head (log2 domain)
+    float l_lane = 0.f;       // this lane's share of the sum of p for head hl
+    float m_run = -INFINITY;  // running max of head hl (log2 domain)
 
     for (int64_t j0 = ja; j0 < jb; j0 += T, ++s) {
       const int slot_i = static_cast<int>(s % kStages);
@@ -423,60 +475,66 @@ __global__ void __launch_bounds__(32 * 9, 1) decode_split_kernel(const DecodeArg
       const int ntok = static_cast<int>(min((int64_t)T, jb - j0));
       const uint8_t* kst = ring + slot_i * L.stage_bytes;
       const uint8_t* vst = kst + T * a.row_bytes;
-      const int head_off = (g * kHeadDim + 8 * c) * ESZ;
 
 #pragma unroll
       for (int sub = 0; sub < T; sub += SUB) {
         if (sub >= ntok) break;
-        // ---- scores: partial dot products over this lane's 8 dims ----------
+        // ---- scores: partial dot products over this lane's units -----------
         float v[V];
 #pragma unroll
-        for (int i = 0; i < HALF; ++i) {
-          const int t = sub + 2 * i + half;
-          float2 k2[4];
-          load8<E>(reinterpret_cast<const E*>(kst + t * a.row_bytes + head_off), k2);
+        for (int i = 0; i < SPL; ++i) {
+          const int t = sub + TL * i + tl;
+          float2 acc[G];
 #pragma unroll
-          for (int hh = 0; hh < G; ++hh) {
-            float2 acc = __fmul2_rn(k2[0], q2[hh][0]);
-            acc = __ffma2_rn(k2[1], q2[hh][1], acc);
-            acc = __ffma2_rn(k2[2], q2[hh][2], acc);
-            acc = __ffma2_rn(k2[3], q2[hh][3], acc);
-            v[hh * HALF + i] = acc.x + acc.y;
+          for (int m = 0; m < UPL; ++m) {
+            float2 k2[4];
+            load8<E>(reinterpret_cast<const E*>(kst + t * a.row_bytes + (g * kHeadDim + 8 * (d + D * m)) * ESZ),
+                     k2);
+#pragma unroll
+            for (int hh = 0; hh < G; ++hh) {
+              acc[hh] = m == 0 ? __fmul2_rn(k2[0], q2[hh][m][0]) : __ffma2_rn(k2[0], q2[hh][m][0], acc[hh]);
+              acc[hh] = __ffma2_rn(k2[1], q2[hh][m][1], acc[hh]);
+              acc[hh] = __ffma2_rn(k2[2], q2[hh][m][2], acc[hh]);
+              acc[hh] = __ffma2_rn(k2[3], q2[hh][m][3], acc[hh]);
+            }
           }
+#pragma unroll
+          for (int hh = 0; hh < G; ++hh) v[hh * SPL + i] = acc[hh].x + acc[hh].y;
         }
-        transpose_reduce16<V>(v, c);
+        transpose_reduce<V, D>(v, d);
         // This lane now holds NV complete scores of head hl.
-        const int idx0 = V >= 16 ? NV * c : (c >> (4 - kLog2V));
-        const int hl = c / LPH;
         float sc[NV];
         float mx = -INFINITY;
 #pragma unroll
         for (int k = 0; k < NV; ++k) {
-          const int idx = idx0 + k;
-          const int tt = 2 * (idx % HALF) + half;
+          const int tt = TL * ((idx0 + k) % SPL) + tl;
           sc[k] = (sub + tt < ntok) ? v[k] : -INFINITY;
           mx = fmaxf(mx, sc[k]);
         }
 #pragma unroll
         for (int off = 1; off < LPH; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+#pragma unroll
+        for (int off = D; off < 32; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
         const bool need = mx > m_run + kRescaleThreshold;
         float alpha = 1.f;
         if (need) {
           alpha = exp2f(m_run - mx);
           m_run = mx;
+          l_lane *= alpha;
         }
 #pragma unroll
         for (int k = 0; k < NV; ++k) {
-          const int idx = idx0 + k;
-          const int tt = 2 * (idx % HALF) + half;
-          pw[tt * G + hl] = exp2f(sc[k] - m_run);
+          const int tt = TL * ((idx0 + k) % SPL) + tl;
+          const float p = exp2f(sc[k] - m_run);
+          if (owner) {
+            pw[tt * G + hl] = p;
+            l_lane += p;
+          }
         }
         if (__any_sync(0xffffffffu, need)) {
 #pragma unroll
           for (int hh = 0; hh < G; ++hh) {
-            const float al = __shfl_sync(0xffffffffu, alpha, hh * LPH);
-            lsum[hh] *= al;
+            const float al = __shfl_sync(0xffffffffu, alpha, head_lane(hh));
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               o2[hh][e].x *= al;
@@ -491,12 +549,12 @@ __global__ void __launch_bounds__(32 * 9, 1) decode_split_kernel(const DecodeArg
           const int tt = 2 * i + half;
           if (sub + tt < ntok) {
             float2 v2[4];
-            load8<E>(reinterpret_cast<const E*>(vst + (sub + tt) * a.row_bytes + head_off), v2);
+            load8<E>(reinterpret_cast<const E*>(vst + (sub + tt) * a.row_bytes + (g * kHeadDim + 8 * c) * ESZ), v2);
+            float p[G];
+            load_p<G>(pw + tt * G, p);
 #pragma unroll
             for (int hh = 0; hh < G; ++hh) {
-              const float p = pw[tt * G + hh];
-              const float2 pp = make_float2(p, p);
-              lsum[hh] += p;
+              const float2 pp = make_float2(p[hh], p[hh]);
 #pragma unroll
               for (int e = 0; e < 4; ++e) o2[hh][e] = __ffma2_rn(v2[e], pp, o2[hh][e]);
             }
@@ -509,9 +567,16 @@ __global__ void __launch_bounds__(32 * 9, 1) decode_split_kernel(const DecodeArg
     }
 
     // ---- finish the piece -----------------------------------------------------
+    // Sum of p per head: the lanes of head hl in every token group.
+#pragma unroll
+    for (int off = 1; off < LPH; off <<= 1) l_lane += __shfl_xor_sync(0xffffffffu, l_lane, off);
+#pragma unroll
+    for (int off = D; off < 32; off <<= 1) l_lane += __shfl_xor_sync(0xffffffffu, l_lane, off);
+    float lsum[G], mh[G];
 #pragma unroll
     for (int hh = 0; hh < G; ++hh) {
-      lsum[hh] += __shfl_xor_sync(0xffffffffu, lsum[hh], 16);
+      lsum[hh] = __shfl_sync(0xffffffffu, l_lane, head_lane(hh));
+      mh[hh] = __shfl_sync(0xffffffffu, m_run, head_lane(hh));
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         o2[hh][e].x += __shfl_xor_sync(0xffffffffu, o2[hh][e].x, 16);
@@ -527,9 +592,6 @@ __global__ void __launch_bounds__(32 * 9, 1) decode_split_kernel(const DecodeArg
           o2[hh][e].y *= a.v_scale;
         }
     }
-    float mh[G];
-#pragma unroll
-    for (int hh = 0; hh < G; ++hh) mh[hh] = __shfl_sync(0xffffffffu, m_run, hh * LPH);
 #pragma unroll
     for (int hh = 0; hh < G; ++hh) {
       if ((G >= 2 ? (hh & 1) : 0) != half) continue;

@@ -16,12 +16,16 @@
 // the V plane).  All arithmetic is fp32; results round to the pool's type.
 #include <cuda_bf16.h>
 
+#include <algorithm>
+
 #include "common.cuh"
 #include "launch.h"
 
 namespace pkv {
 
 namespace {
+
+constexpr int64_t kSmCountHint = 148;  // B200
 
 struct RopeArgs {
   uint8_t* kpool;
@@ -93,10 +97,14 @@ __device__ __forceinline__ void load_w8(const void* w, int c, float (&f)[8]) {
   }
 }
 
-// One block per token.  Its kThreads / 16 half-warps walk the token's head
-// rows with that stride, kRif rows at a time: every row load of a group is
-// issued before any of them is used, and the token's position, slot and
-// cos/sin values are loaded once per half-warp, not once per row.
+// Block (token, row group).  The kThreads / 16 half-warps of a block walk the
+// token's head rows kRif at a time (every row load of a group is issued
+// before any of them is used), starting at row group blockIdx.y; the
+// gridDim.y blocks of a token interleave their groups.  The token's position,
+// slot and cos/sin values are loaded once per half-warp, not once per row.
+// Large batches use gridDim.y = 1 (one block walks all rows of a token); small
+// ones (a decode step) split a token's rows over several blocks so that every
+// row load is in flight at once.
 // kFp8: the pool holds E4M3 codes; k and v rows are stored as the codes of
 // value * (1 / scale) (E is then bf16, the type of qkv and q_out).
 template <typename E, int kThreads, int kRif, int kMinBlocks, bool kFp8>
@@ -108,12 +116,15 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) qk_norm_rope_store_kerne
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int64_t t = blockIdx.x;
   const int rows = a.hq + 2 * a.hkv;
-  const int hw = threadIdx.x >> 4;  // half-warp: the first row it owns
+  const int hw = threadIdx.x >> 4;  // half-warp within the block
+  constexpr int kGroupRows = kHalfWarps * kRif;
+  const int rfirst = hw + static_cast<int>(blockIdx.y) * kGroupRows;  // first row it owns
+  const int rstride = kGroupRows * static_cast<int>(gridDim.y);
   const int c = threadIdx.x & 15;   // 8-element chunk of a head row
   // The 16 lanes of a half-warp follow the same path; the two halves of a
   // warp may not (different row kinds), so every shuffle stays in its half.
   const unsigned hmask = (threadIdx.x & 16) ? 0xffff0000u : 0x0000ffffu;
-  if (hw >= rows) return;  // whole half-warps only
+  if (rfirst >= rows) return;  // whole half-warps only
 
   const int64_t pos = a.pos_i64 ? static_cast<const int64_t*>(a.positions)[t]
                                 : static_cast<int64_t>(static_cast<const int32_t*>(a.positions)[t]);
@@ -121,7 +132,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) qk_norm_rope_store_kerne
                                  : static_cast<int64_t>(static_cast<const int32_t*>(a.out_loc)[t]);
   const bool pos_ok = pos >= 0 && pos < a.max_position;
   const bool slot_ok = slot >= 0 && slot < a.num_slots;
-  if (threadIdx.x == 0) {
+  if (threadIdx.x == 0 && blockIdx.y == 0) {
     if (!pos_ok) set_err(a.err, PKV_DEV_ERR_POSITION);
     if (!slot_ok) set_err(a.err, PKV_DEV_ERR_SLOT_RANGE);
   }
@@ -140,7 +151,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) qk_norm_rope_store_kerne
   }
   const float sign = (c < 8) ? -1.f : 1.f;  // x1 cos - x2 sin | x2 cos + x1 sin
 
-  for (int r0 = hw; r0 < rows; r0 += kHalfWarps * kRif) {
+  for (int r0 = rfirst; r0 < rows; r0 += rstride) {
     Chunk8<E> raw[kRif];
 #pragma unroll
     for (int u = 0; u < kRif; ++u) {
@@ -230,10 +241,19 @@ cudaError_t launch_qk_norm_rope_store(const PoolView& pool, const void* qkv, int
   a.q_out = q_out;
   a.err = err;
   if (n > 0x7fffffffLL) return cudaErrorInvalidValue;
-  const unsigned blocks = static_cast<unsigned>(n);
   // 64-thread blocks (4 half-warps, 4 rows in flight each) at 16 blocks per
   // SM: measured best on B200 among 32-512 threads and 2-8 rows in flight
-  // (about 96% of copy bandwidth at 32k tokens of Hq 32 / Hkv 8).
+  // (about 96% of copy bandwidth at 32k tokens of Hq 32 / Hkv 8).  Below
+  // about four blocks per SM the rows of a token are split over row groups
+  // (blockIdx.y), so that a decode step's few tokens put all their row loads
+  // in flight in one pass instead of walking them one group after another.
+  const int rif = pool.dtype == PKV_DTYPE_F32 ? 2 : 4;
+  const int64_t rows = num_q_heads + 2LL * pool.num_kv_heads;
+  const int64_t groups = (rows + 4 * rif - 1) / (4 * rif);
+  const int64_t want = 4LL * kSmCountHint;
+  int64_t ysplit = 1;
+  if (n < want) ysplit = std::min<int64_t>(groups, (want + n - 1) / n);
+  const dim3 blocks(static_cast<unsigned>(n), static_cast<unsigned>(ysplit));
   a.k_inv = 1.0f / pool.k_scale;
   a.v_inv = 1.0f / pool.v_scale;
   if (pool.dtype == PKV_DTYPE_BF16)

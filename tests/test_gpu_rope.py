@@ -157,6 +157,21 @@ def test_rope_store_position_edges():
     _compare(wl, dev)
 
 
+@pytest.mark.parametrize("n,hq,hkv", [(64, 16, 8), (256, 32, 8), (64, 64, 8), (1000, 32, 8)])
+def test_rope_store_launch_shapes(n, hq, hkv):
+    """Both launch shapes: decode-sized batches split every token's rows over
+    several blocks (64 and 256 tokens, the decode steps of the Qwen3-0.6B and
+    Qwen3-8B shapes), large batches walk a token's rows in one block."""
+    rng = np.random.default_rng(100 + n + hq)
+    pos = rng.integers(0, 8192, size=n).astype(np.int32)
+    wl = W.rope_store_step(W.BF16, positions=pos, num_q_heads=hq, num_kv_heads=hkv,
+                           num_slots=max(4096, 2 * n), seed=200 + n + hq)
+    dev = DevRope(wl)
+    dev.run()
+    assert int(dev.err.item()) == 0
+    _compare(wl, dev)
+
+
 def test_rope_store_bad_position_zeroes_and_flags():
     maxp = 1024
     pos = np.array([3, maxp, 7, -1, 500], dtype=np.int32)
