@@ -337,6 +337,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     set_err(a.err, PKV_DEV_ERR_BAD_LENGTH);
   const int i0 = qb * (kQTiles * TQ);
   if (i0 >= e) return;
+  // Q tile 1 holds a valid token only if the block has more than TQ of them;
+  // otherwise (the last block of a short chunk) its MMAs and softmax are skipped.
+  const bool tile1 = i0 + TQ < e;
   // Prefix mode reads the keys through the row of the group's first member.
   const int32_t trow = a.table_idx[a.prefix_mode ? qbase : r];
   const bool row_ok = trow >= 0 && trow < a.table_rows;
@@ -570,7 +573,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       tc_fence_after();
       issue_qk(0, j);
-      issue_qk(1, j);
+      if (tile1) issue_qk(1, j);
       commit(kBarKEmpty + j);
     }
     for (int j = 0; j < nsteps && ok; ++j) {
@@ -587,13 +590,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         issue_qk(0, j + 2);
       }
-      ok = wait_all(kBarPReady + 2 + (j & 1), (j >> 1) & 1);
-      if (!ok || __any_sync(0xffffffffu, *abort_flag != 0)) break;
-      tc_fence_after();
-      issue_pv(1, j);
+      if (tile1) {
+        ok = wait_all(kBarPReady + 2 + (j & 1), (j >> 1) & 1);
+        if (!ok || __any_sync(0xffffffffu, *abort_flag != 0)) break;
+        tc_fence_after();
+        issue_pv(1, j);
+      }
       commit(kBarVEmpty + st);
       if (more) {
-        issue_qk(1, j + 2);
+        if (tile1) issue_qk(1, j + 2);
         commit(kBarKEmpty + st2);
       }
     }
@@ -638,7 +643,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       mbar_arrive(&bars[kBarQReady]);
     }
-    for (int j = 0; j < nsteps; ++j) {
+    const int my_steps = (i == 0 || tile1) ? nsteps : 0;  // tile 1 may have no valid row
+    for (int j = 0; j < my_steps; ++j) {
       const int hf = j & 1;
       const uint32_t s_addr = tmem + lane_base + kColS + 128 * i + 64 * hf;
       const bool w = mbar_wait(&bars[kBarSFull + 2 * i + hf], (j >> 1) & 1);

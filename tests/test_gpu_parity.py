@@ -268,6 +268,7 @@ def test_extend_group_sizes(dtype, hq, hkv):
     d.run()
     exp, _ = oracle_extend(wl)
     tol_check(from_dev(d.out), exp, dtype, f"extend hq={hq} hkv={hkv}")
+    assert _err(d.err) == 0
 
 
 def test_extend_zero_length_requests_in_batch():
@@ -276,6 +277,23 @@ def test_extend_zero_length_requests_in_batch():
     d.run()
     exp, _ = oracle_extend(wl)
     tol_check(from_dev(d.out), exp, W.BF16, "extend with empty chunks")
+    assert _err(d.err) == 0
+
+
+def test_extend_ragged_batch_of_40():
+    """40 requests with chunks of 1..299 tokens after prefixes of 0..899: short
+    last query blocks (whose second Q tile holds no token and is skipped),
+    diagonal steps at every offset, every row compared."""
+    rng = np.random.default_rng(77)
+    ext = rng.integers(1, 300, size=40)
+    pre = rng.integers(0, 900, size=40)
+    wl = W.extend_small(prefix_lens=tuple(int(x) for x in pre), extend_lens=tuple(int(x) for x in ext),
+                        num_q_heads=32, num_kv_heads=8, num_slots=int((pre + ext).sum()) + 64, seed=1500)
+    d = DeviceExtend(wl)
+    d.run()
+    exp, _ = oracle_extend(wl)
+    tol_check(from_dev(d.out), exp, W.BF16, "extend, 40 ragged requests")
+    assert _err(d.err) == 0
 
 
 def _chunk_rows(prefix: int, e: int, hq: int, hkv: int, seed: int):
