@@ -49,7 +49,7 @@ sys.path.insert(0, ROOT)
 
 HBM_FALLBACK_GBS = 6650.0
 BF16_FALLBACK_TFLOPS = 1590.0
-NORTH_STAR_HBM_GBS = 8000.0  # the ~8 TB/s nominal figure decode is also reported against
+NOMINAL_HBM_GBS = 8000.0  # B200 nominal HBM3e bandwidth; decode is also reported against it
 
 
 # ---------------------------------------------------------------------------
@@ -541,7 +541,7 @@ def run_decode(args, world, rank, local, name):
             "peak_source": peak_src,
             "unit": "GB/s",
             "frac": round(achieved / hbm, 4),
-            "frac_of_8tbs": round(achieved / NORTH_STAR_HBM_GBS, 4),
+            "frac_of_8tbs": round(achieved / NOMINAL_HBM_GBS, 4),
             "traffic": traffic,
             "algorithmic_bytes_per_launch": per_call,
         },
