@@ -35,7 +35,12 @@
 //  * FP8 (E4M3) pools: 32 tokens per stage (1 KB rows); codes widen exactly to
 //    half and then float; the K scale is folded into the softmax scale and
 //    the V scale into the output.
+#include <cuda.h>
 #include <cuda_bf16.h>
+#include <cudaTypedefs.h>
+
+#include <cstring>
+#include <type_traits>
 
 #include "common.cuh"
 #include "launch.h"
@@ -98,25 +103,112 @@ struct DecodeArgs {
   int32_t cascade;
 };
 
-// Shared memory layout (bytes), identical on host and device.
+// Shared memory layout (bytes), identical on host and device.  A stage holds
+// T K rows then T V rows, row_stride bytes apart.
 struct DecodeSmem {
   int32_t cum_off, psm_off, ring_off, stage_bytes, total;
 };
 
-__host__ __device__ inline DecodeSmem decode_smem_layout(int batch, int hkv, int row_bytes, int T,
-                                                         int G) {
+__host__ __device__ inline DecodeSmem decode_smem_layout(int batch, int hkv, int row_stride, int T,
+                                                         int psm_per_warp) {
   DecodeSmem L;
   int off = 2 * kStages * 8 + 16;  // full/empty barriers + abort flag
   L.cum_off = off;
   off += 4 * (batch + 1);
   off = (off + 15) & ~15;
   L.psm_off = off;
-  off += 4 * hkv * T * G;
-  off = (off + 127) & ~127;
+  off += hkv * psm_per_warp;
+  off = (off + 1023) & ~1023;  // page boxes are 128B-swizzled: 1024-byte aligned
   L.ring_off = off;
-  L.stage_bytes = 2 * T * row_bytes;
+  L.stage_bytes = 2 * T * row_stride;
   L.total = off + kStages * L.stage_bytes;
   return L;
+}
+
+// Tensor-core consumers (bf16 and FP8 pools) read the ring with ldmatrix,
+// eight rows of 16 bytes per matrix.  A 16-byte pad after every row (rows are
+// a multiple of 128 bytes) puts those eight rows in eight different bank
+// groups.
+template <typename E>
+struct DecodeLayoutTraits {
+  static constexpr bool kMma = sizeof(E) != 4;
+  static constexpr int kRowPad = kMma ? 16 : 0;
+  static constexpr int kPStride = 40;  // p buffer row (16-bit entries) per head, 32 tokens + pad
+  template <int G>
+  static constexpr int psm_per_warp() {
+    return kMma ? 8 * kPStride * 2 : 4 * DecodeTraits<E>::kTokensPerStage * G;
+  }
+};
+
+// ---- mma.sync helpers (m16n8k16, fp32 accumulate) -----------------------------
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+
+// c += A (16 x 16, row-major fragment) * B (16 x 8, column-major fragment);
+// A and B both bf16 (kF16 = false) or both f16.
+template <bool kF16>
+__device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  if constexpr (kF16) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+  } else {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+  }
+}
+
+// The two E4M3 codes in the low (lo_f16x2) or high (hi_f16x2) half of w, low
+// byte first -> f16x2, exact.
+__device__ __forceinline__ uint32_t lo_f16x2(uint32_t w) {
+  uint32_t r;
+  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, l;\n\t}" : "=r"(r) : "r"(w));
+  return r;
+}
+__device__ __forceinline__ uint32_t hi_f16x2(uint32_t w) {
+  uint32_t r;
+  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, h;\n\t}" : "=r"(r) : "r"(w));
+  return r;
+}
+
+// One page box (16 slots from `slot`, every KV head) of a pool plane into a
+// stage: a 4-D map (64 elements, slot, half row, head) for bf16 rows, a 3-D
+// map (128 codes, slot, head) for E4M3 rows; see make_page_map.
+template <typename E>
+__device__ __forceinline__ void tma_page_box(void* dst, const CUtensorMap* map, int32_t slot, uint64_t* bar,
+                                             uint64_t policy) {
+  if constexpr (sizeof(E) == 1) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(smem_u32(dst)),
+        "l"(map), "r"(0), "r"(slot), "r"(0), "r"(smem_u32(bar)), "l"(policy)
+        : "memory");
+  } else {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%2, %3, %4, %5}], [%6], %7;" ::"r"(smem_u32(dst)),
+        "l"(map), "r"(0), "r"(slot), "r"(0), "r"(0), "r"(smem_u32(bar)), "l"(policy)
+        : "memory");
+  }
+}
+
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  const __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
 }
 
 // Transposing butterfly over groups of D consecutive lanes (D = 8 or 16).  On
@@ -185,8 +277,13 @@ __device__ __forceinline__ void load_p(const float* src, float (&p)[G]) {
   }
 }
 
-template <typename E, int G>
-__global__ void __launch_bounds__(32 * 9, 1) decode_split_kernel(const DecodeArgs a) {
+// kPaged: the pool's page size is a multiple of 16 and each ring stage is
+// loaded as page boxes (one tensor copy per plane per 16 table columns)
+// through kmap / vmap; otherwise one bulk copy per token row per plane.
+template <typename E, int G, bool kPaged>
+__global__ void __launch_bounds__(32 * 9, 1) decode_split_kernel(const DecodeArgs a,
+                                                                 const __grid_constant__ CUtensorMap kmap,
+                                                                 const __grid_constant__ CUtensorMap vmap) {
   constexpr int T = DecodeTraits<E>::kTokensPerStage;
   constexpr int SUB = (64 / G < T) ? 64 / G : T;  // tokens per softmax sub-step
   constexpr int HALF = SUB / 2;                    // PV: tokens per lane per sub-step
@@ -211,12 +308,18 @@ __global__ void __launch_bounds__(32 * 9, 1) decode_split_kernel(const DecodeArg
   using IO = typename DecodeTraits<E>::IO;
   static_assert(SUB % TL == 0 && NV <= SPL, "decode sub-step shape");
 
-  extern __shared__ __align__(128) uint8_t smem[];
+  extern __shared__ __align__(128) uint8_t smem_raw[];
+  // Page-box stages need 1024-byte alignment (the host adds 1 KB of slack).
+  uint8_t* smem = kPaged ? reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023))
+                         : smem_raw;
   // Let the combine kernel be scheduled early; it waits for this grid anyway.
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int ncons = a.hkv;
-  const DecodeSmem L = decode_smem_layout(a.batch, a.hkv, a.row_bytes, T, G);
+  using LT = DecodeLayoutTraits<E>;
+  static_assert(!kPaged || LT::kMma, "page-box stages feed the tensor-core consumers");
+  const int RS = a.row_bytes + (kPaged ? 0 : LT::kRowPad);  // ring row stride
+  const DecodeSmem L = decode_smem_layout(a.batch, a.hkv, RS, T, LT::template psm_per_warp<G>());
   uint64_t* full = reinterpret_cast<uint64_t*>(smem);
   uint64_t* empty = full + kStages;
   volatile int32_t* abort_flag = reinterpret_cast<volatile int32_t*>(empty + kStages);
@@ -298,6 +401,142 @@ __global__ void __launch_bounds__(32 * 9, 1) decode_split_kernel(const DecodeArg
   }
 
   if (warp == 0) {
+    if constexpr (kPaged) {
+      // ====================== producer (page boxes) ===========================
+      // A stage is NG groups of 16 table columns aligned to 16.  Each group
+      // lies inside one page (the page size is a multiple of 16), so it is one
+      // tensor copy per plane: 16 consecutive slots of every KV head, which
+      // lands 128B-swizzled as [head][half][slot][128 B] (bf16) or
+      // [head][slot][128 B] (FP8).  Rows of a group outside the piece are
+      // loaded too and masked by the consumers.  Lane n < NG owns group n;
+      // table entries are loaded two stages ahead.
+      constexpr int NG = T / 16;
+      const int box_bytes = 16 * a.row_bytes;
+      const uint64_t policy = policy_evict_first();
+      struct Cursor {
+        int r;
+        int64_t j0, jb;  // piece tokens [j0, jb) of the pass, relative to col0
+        int32_t col0;    // table column of the pass's token 0
+        const int32_t* rowp;
+        bool row_ok;
+      };
+      auto piece_start = [&](int rr, Cursor& c) -> bool {
+        for (; rr < B && cum[rr] < hi; ++rr) {
+          const int64_t ja = max(lo, (int64_t)cum[rr]) - cum[rr];
+          const int64_t jb = min(hi, (int64_t)cum[rr + 1]) - cum[rr];
+          if (jb > ja) {
+            const int32_t trow = a.table_idx[rr];
+            c.row_ok = trow >= 0 && trow < a.table_rows;
+            if (!c.row_ok && lane == 0) set_err(a.err, PKV_DEV_ERR_TABLE_RANGE);
+            c.rowp = a.table + (c.row_ok ? trow : 0) * a.table_stride;
+            c.col0 = a.kv_start != nullptr ? max(a.kv_start[rr], 0) : 0;
+            c.r = rr;
+            c.j0 = ja;
+            c.jb = jb;
+            return true;
+          }
+        }
+        return false;
+      };
+      // End column (exclusive) of the stage that starts at the cursor.
+      auto stage_end = [&](const Cursor& c) -> int64_t {
+        const int64_t cs = c.col0 + c.j0;
+        return min((int64_t)c.col0 + c.jb, (cs & ~int64_t(15)) + 16 * NG);
+      };
+      auto advance = [&](Cursor& c) -> bool {
+        const int64_t ce = stage_end(c);
+        if (ce < (int64_t)c.col0 + c.jb) {
+          c.j0 = ce - c.col0;
+          return true;
+        }
+        return piece_start(c.r + 1, c);
+      };
+      // First table column of this lane's group of the stage at the cursor.
+      auto group_col = [&](const Cursor& c) -> int64_t {
+        return ((c.col0 + c.j0) & ~int64_t(15)) + 16 * lane;
+      };
+      // This lane's raw table entry (its group's page's first slot).
+      auto lookup = [&](const Cursor& c, bool have) -> int32_t {
+        if (!have || lane >= NG || !c.row_ok) return 0;
+        const int64_t col = group_col(c);
+        if (col >= stage_end(c)) return 0;
+        const int32_t c32 = static_cast<int32_t>(col);
+        return c.rowp[c32 - page_offset(c32, a.page_size)];
+      };
+      Cursor c0{}, c1{}, c2{};
+      bool h0 = piece_start(rfirst, c0);
+      int32_t e0 = lookup(c0, h0);
+      c1 = c0;
+      bool h1 = h0 && advance(c1);
+      int32_t e1 = lookup(c1, h1);
+      c2 = c1;
+      bool h2 = h1 && advance(c2);
+      int last_use[kStages];
+#pragma unroll
+      for (int i = 0; i < kStages; ++i) last_use[i] = -1;
+      for (int64_t s = 0; h0; ++s) {
+        const int32_t e2 = lookup(c2, h2);
+        const int slot_i = static_cast<int>(s % kStages);
+        const int use = static_cast<int>(s / kStages);
+        if (use >= 1) {
+          bool ok = true;
+          if (lane == 0) ok = mbar_wait(&empty[slot_i], (use - 1) & 1);
+          ok = __shfl_sync(0xffffffffu, ok, 0);
+          if (__any_sync(0xffffffffu, !ok || *abort_flag != 0)) {
+            if (!ok && lane == 0) set_err(a.err, PKV_DEV_ERR_TIMEOUT);
+            *abort_flag = 1;
+            break;
+          }
+        }
+        uint8_t* kst = ring + slot_i * L.stage_bytes;
+        uint8_t* vst = kst + NG * box_bytes;
+        const int64_t col = group_col(c0);
+        const bool in_stage = lane < NG && col < stage_end(c0);
+        int32_t slot = -1;
+        if (in_stage && c0.row_ok) {
+          if (page_offset(e0, a.page_size) != 0) {
+            set_err(a.err, PKV_DEV_ERR_PAGE_ALIGN);
+          } else {
+            const int64_t sl = static_cast<int64_t>(e0) + page_offset(static_cast<int32_t>(col), a.page_size);
+            if (sl < 0 || sl >= a.num_slots)
+              set_err(a.err, PKV_DEV_ERR_SLOT_RANGE);
+            else
+              slot = static_cast<int32_t>(sl);
+          }
+        }
+        const bool load = in_stage && slot >= 0;
+        if (in_stage && !load) {
+          // Bad entry: the group reads as zeros (error already flagged).
+          for (int b = 0; b < box_bytes; b += 16) {
+            *reinterpret_cast<uint4*>(kst + lane * box_bytes + b) = make_uint4(0, 0, 0, 0);
+            *reinterpret_cast<uint4*>(vst + lane * box_bytes + b) = make_uint4(0, 0, 0, 0);
+          }
+          // Later tensor copies (async proxy) may write these bytes again.
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        }
+        const unsigned nload = __popc(__ballot_sync(0xffffffffu, load));
+        __syncwarp();
+        if (lane == 0) mbar_arrive_expect_tx(&full[slot_i], nload * 2u * box_bytes);
+        __syncwarp();
+        if (load) {
+          tma_page_box<E>(kst + lane * box_bytes, &kmap, slot, &full[slot_i], policy);
+          tma_page_box<E>(vst + lane * box_bytes, &vmap, slot, &full[slot_i], policy);
+        }
+        last_use[slot_i] = use;
+        c0 = c1;
+        h0 = h1;
+        e0 = e1;
+        c1 = c2;
+        h1 = h2;
+        e1 = e2;
+        if (h2) h2 = advance(c2);
+      }
+      if (lane == 0) {
+        for (int i = 0; i < kStages; ++i)
+          if (last_use[i] >= 0 && !mbar_wait(&full[i], last_use[i] & 1))
+            set_err(a.err, PKV_DEV_ERR_TIMEOUT);
+      }
+    } else {
     // =========================== producer ===================================
     // Page-table entries are loaded two stages ahead of the copies that use
     // them, so the dependent table read overlaps the wait for a free stage.
@@ -368,7 +607,7 @@ __global__ void __launch_bounds__(32 * 9, 1) decode_split_kernel(const DecodeArg
         }
       }
       uint8_t* kst = ring + slot_i * L.stage_bytes;
-      uint8_t* vst = kst + T * a.row_bytes;
+      uint8_t* vst = kst + T * RS;
       const int64_t j = c0.j0 + lane;
       const bool in_piece = lane < T && j < c0.jb;
       int64_t slot = -1;
@@ -391,8 +630,8 @@ __global__ void __launch_bounds__(32 * 9, 1) decode_split_kernel(const DecodeArg
       if (in_piece && !load) {
         // Out-of-range entry: the row reads as zeros (error already flagged).
         for (int b = 0; b < a.row_bytes; b += 16) {
-          *reinterpret_cast<uint4*>(kst + lane * a.row_bytes + b) = make_uint4(0, 0, 0, 0);
-          *reinterpret_cast<uint4*>(vst + lane * a.row_bytes + b) = make_uint4(0, 0, 0, 0);
+          *reinterpret_cast<uint4*>(kst + lane * RS + b) = make_uint4(0, 0, 0, 0);
+          *reinterpret_cast<uint4*>(vst + lane * RS + b) = make_uint4(0, 0, 0, 0);
         }
         // Later bulk copies (async proxy) may write these bytes again.
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -402,9 +641,9 @@ __global__ void __launch_bounds__(32 * 9, 1) decode_split_kernel(const DecodeArg
       if (lane == 0) mbar_arrive_expect_tx(&full[slot_i], nload * 2u * a.row_bytes);
       __syncwarp();
       if (load) {
-        bulk_g2s(kst + lane * a.row_bytes, a.kbase + slot * a.slot_stride_bytes, a.row_bytes,
+        bulk_g2s(kst + lane * RS, a.kbase + slot * a.slot_stride_bytes, a.row_bytes,
                  &full[slot_i], policy);
-        bulk_g2s(vst + lane * a.row_bytes, a.vbase + slot * a.slot_stride_bytes, a.row_bytes,
+        bulk_g2s(vst + lane * RS, a.vbase + slot * a.slot_stride_bytes, a.row_bytes,
                  &full[slot_i], policy);
       }
       last_use[slot_i] = use;
@@ -423,9 +662,375 @@ __global__ void __launch_bounds__(32 * 9, 1) decode_split_kernel(const DecodeArg
         if (last_use[i] >= 0 && !mbar_wait(&full[i], last_use[i] & 1))
           set_err(a.err, PKV_DEV_ERR_TIMEOUT);
     }
+    }
     return;
   }
 
+  if constexpr (LT::kMma) {
+    // ======================= consumers (tensor cores) =========================
+    // Per 16-token sub-step, with the GQA group as the N dimension:
+    //   S^T (16 tokens x 8 heads)  = K (16 x 128) . Q^T (128 x 8)  8 MMAs
+    //   O^T (128 dims x 8 heads)  += V^T (128 x 16) . P^T (16 x 8)  8 MMAs
+    // Lane (qr, kq) = (lane / 4, lane % 4) holds scores of tokens qr, qr + 8
+    // and output columns for heads 2kq, 2kq + 1 (columns >= G are padding),
+    // so its softmax state (max, sum) covers exactly the heads whose output it
+    // accumulates.  P passes from the score layout to the PV B fragment
+    // through the warp's p buffer [head][token] (16-bit).  bf16 pools run bf16
+    // MMAs on the stored rows; FP8 pools widen codes exactly to f16 and run
+    // f16 MMAs (q enters as f16 scaled by 2^-8, undone in the score scale).
+    constexpr bool kF8 = sizeof(E) == 1;
+    constexpr int NT = T / 16;  // 16-token tiles per stage (bf16 1, FP8 2)
+    constexpr int kPS = LT::kPStride;
+    static_assert(T == 16 * NT, "decode tensor-core stage");
+    constexpr float kQPre = kF8 ? 1.f / 256.f : 1.f;
+    const int g = warp - 1;  // KV head
+    if (g >= ncons) return;
+    const int qr = lane >> 2, kq = lane & 3;
+    const bool v0 = 2 * kq < G, v1 = 2 * kq + 1 < G;
+    const float sl = kF8 ? a.scale_log2 * 256.f : a.scale_log2;
+    uint16_t* pw = reinterpret_cast<uint16_t*>(smem + L.psm_off) + g * (8 * kPS);
+    const uint32_t ring_s = smem_u32(ring);
+    // ldmatrix row of this lane: K (plain) matrices are (tokens 0-7 | 8-15) x
+    // (first | second 16 bytes); V (transposed) matrices are (first | second
+    // 16 bytes) x (tokens 0-7 | 8-15).
+    const int tok_k = (lane & 7) + ((lane >> 3) & 1) * 8, col_k = lane >> 4;
+    const int tok_v = (lane & 7) + (lane >> 4) * 8, col_v = (lane >> 3) & 1;
+    const int x7 = lane & 7;
+    const int box_bytes = 16 * a.row_bytes;  // one page box: 16 slots of all KV heads
+    const IO* qbase = static_cast<const IO*>(a.q);
+    IO* obase = static_cast<IO*>(a.out);
+    int64_t s = 0;
+    for (int r = rfirst; r < B && cum[r] < hi; ++r) {
+      const int64_t ja = max(lo, (int64_t)cum[r]) - cum[r];
+      const int64_t jb = min(hi, (int64_t)cum[r + 1]) - cum[r];
+      if (jb <= ja) continue;
+      const bool whole = !a.cascade && cum[r] >= lo && cum[r + 1] <= hi;
+      if (r + 1 < B && cum[r + 1] < hi && lane < 2 * G)
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(qbase + ((int64_t)(r + 1) * a.hq + g * G) * kHeadDim +
+                                                        lane * (128 / static_cast<int>(sizeof(IO)))));
+      // Q^T B fragments, 16 dims per MMA: b0 = dims k, k + 1 and b1 = dims
+      // k + 8, k + 9 (k = 2 kq) of head qr.  FP8 rows use the dim order of
+      // their K fragments instead: b0 = dims 4kq, 4kq + 1, b1 = 4kq + 2, 4kq + 3.
+      uint32_t qb[8][2];
+      if (qr < G) {
+        const IO* qrow = qbase + ((int64_t)r * a.hq + g * G + qr) * kHeadDim;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          if constexpr (kF8) {
+            const uint2 w = *reinterpret_cast<const uint2*>(qrow + 16 * c + 4 * kq);
+            qb[c][0] = pack_f16x2(bf16_lo(w.x) * kQPre, bf16_hi(w.x) * kQPre);
+            qb[c][1] = pack_f16x2(bf16_lo(w.y) * kQPre, bf16_hi(w.y) * kQPre);
+          } else {
+            qb[c][0] = *reinterpret_cast<const uint32_t*>(qrow + 16 * c + 2 * kq);
+            qb[c][1] = *reinterpret_cast<const uint32_t*>(qrow + 16 * c + 2 * kq + 8);
+          }
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < 8; ++c) qb[c][0] = qb[c][1] = 0u;
+      }
+      float acc[8][4];
+#pragma unroll
+      for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[mt][e] = 0.f;
+      float l0 = 0.f, l1 = 0.f;              // this lane's share of the sums of p
+      float m0 = -INFINITY, m1 = -INFINITY;  // running max of heads 2kq, 2kq + 1 (log2 domain)
+
+      // Stages: T tokens each (row copies), or NT groups of 16 table columns
+      // aligned to 16 (page boxes; a piece's first and last groups may be
+      // partial).  Tile nt of a stage holds its valid tokens at box rows
+      // [lo_t[nt], hi_t[nt]).
+      const int32_t col0 = (kPaged && a.kv_start != nullptr) ? max(a.kv_start[r], 0) : 0;
+      int64_t j0 = ja;
+      while (j0 < jb) {
+        const int slot_i = static_cast<int>(s % kStages);
+        const int use = static_cast<int>(s / kStages);
+        bool ok = mbar_wait(&full[slot_i], use & 1);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok || *abort_flag) {
+          if (!ok && lane == 0) set_err(a.err, PKV_DEV_ERR_TIMEOUT);
+          *abort_flag = 1;
+          return;
+        }
+        int lo_t[NT], hi_t[NT];
+        int64_t jn;
+        if constexpr (kPaged) {
+          const int64_t cs = col0 + j0, b0 = cs & ~int64_t(15);
+          const int64_t ce = min((int64_t)col0 + jb, b0 + 16 * NT);
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) {
+            lo_t[nt] = static_cast<int>(max(cs - (b0 + 16 * nt), (int64_t)0));
+            hi_t[nt] = static_cast<int>(min(ce - (b0 + 16 * nt), (int64_t)16));
+          }
+          jn = ce - col0;
+        } else {
+          const int ntok = static_cast<int>(min((int64_t)T, jb - j0));
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) {
+            lo_t[nt] = 0;
+            hi_t[nt] = min(16, ntok - 16 * nt);
+          }
+          jn = j0 + T;
+        }
+        const uint32_t kst = ring_s + slot_i * L.stage_bytes;
+        const uint32_t vst = kst + T * RS;  // T * row_bytes in page-box stages
+        // ldmatrix row addresses of 16-dim chunk c (bf16) or 16-code chunk
+        // pair cp (FP8) of tile nt: padded rows, or 128B-swizzled page boxes
+        // [head][half (bf16)][16 slots][128 B] (16-byte chunk x of box row t
+        // stored at chunk x ^ (t & 7); here t & 7 = lane & 7).
+        auto k_addr = [&](int nt, int c) -> uint32_t {
+          if constexpr (kPaged) {
+            if constexpr (kF8)
+              return kst + nt * box_bytes + (g * 16 + tok_k) * 128 + (((2 * c + col_k) ^ x7) << 4);
+            else
+              return kst + nt * box_bytes + ((g * 2 + (c >> 2)) * 16 + tok_k) * 128 +
+                     ((((2 * c + col_k) & 7) ^ x7) << 4);
+          } else {
+            if constexpr (kF8)
+              return kst + (16 * nt + tok_k) * RS + g * kHeadDim + 16 * (2 * c + col_k);
+            else
+              return kst + (16 * nt + tok_k) * RS + (g * kHeadDim + 16 * c + 8 * col_k) * 2;
+          }
+        };
+        auto v_addr = [&](int nt, int c) -> uint32_t {
+          if constexpr (kPaged) {
+            if constexpr (kF8)
+              return vst + nt * box_bytes + (g * 16 + tok_v) * 128 + (((2 * c + col_v) ^ x7) << 4);
+            else
+              return vst + nt * box_bytes + ((g * 2 + (c >> 2)) * 16 + tok_v) * 128 +
+                     ((((2 * c + col_v) & 7) ^ x7) << 4);
+          } else {
+            if constexpr (kF8)
+              return vst + (16 * nt + tok_v) * RS + g * kHeadDim + 16 * (2 * c + col_v);
+            else
+              return vst + (16 * nt + tok_v) * RS + (g * kHeadDim + 16 * c + 8 * col_v) * 2;
+          }
+        };
+        // ---- scores: NT independent 16-token tiles, each with two
+        // accumulators (even and odd 16-dim chunks) to halve the MMA chain.
+        float sc[NT][4];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          float se[4] = {0.f, 0.f, 0.f, 0.f}, so[4] = {0.f, 0.f, 0.f, 0.f};
+          if (hi_t[nt] > lo_t[nt]) {
+            if constexpr (kF8) {
+#pragma unroll
+              for (int cp = 0; cp < 4; ++cp) {
+                uint32_t w[4];
+                ldsm_x4(k_addr(nt, cp), w);
+                // w[0], w[1]: tokens 0-7, 8-15 of 16-dim chunk 2cp; w[2], w[3]: chunk 2cp + 1.
+                const uint32_t f0[4] = {lo_f16x2(w[0]), lo_f16x2(w[1]), hi_f16x2(w[0]), hi_f16x2(w[1])};
+                const uint32_t f1[4] = {lo_f16x2(w[2]), lo_f16x2(w[3]), hi_f16x2(w[2]), hi_f16x2(w[3])};
+                mma16816<true>(se, f0, qb[2 * cp][0], qb[2 * cp][1]);
+                mma16816<true>(so, f1, qb[2 * cp + 1][0], qb[2 * cp + 1][1]);
+              }
+            } else {
+#pragma unroll
+              for (int c = 0; c < 8; c += 2) {
+                uint32_t f0[4], f1[4];
+                ldsm_x4(k_addr(nt, c), f0);
+                ldsm_x4(k_addr(nt, c + 1), f1);
+                mma16816<false>(se, f0, qb[c][0], qb[c][1]);
+                mma16816<false>(so, f1, qb[c + 1][0], qb[c + 1][1]);
+              }
+            }
+          }
+#pragma unroll
+          for (int e = 0; e < 4; ++e) sc[nt][e] = se[e] + so[e];
+        }
+        // sc[nt] = S[token qr][head 2kq], S[qr][2kq + 1], S[qr + 8][2kq],
+        // S[qr + 8][2kq + 1] of tile nt; scaled to the log2 domain, masked.
+        float sv[NT][4];
+        float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          const bool t0 = qr >= lo_t[nt] && qr < hi_t[nt];
+          const bool t1 = qr + 8 >= lo_t[nt] && qr + 8 < hi_t[nt];
+          sv[nt][0] = (v0 && t0) ? sc[nt][0] * sl : -INFINITY;
+          sv[nt][1] = (v1 && t0) ? sc[nt][1] * sl : -INFINITY;
+          sv[nt][2] = (v0 && t1) ? sc[nt][2] * sl : -INFINITY;
+          sv[nt][3] = (v1 && t1) ? sc[nt][3] * sl : -INFINITY;
+          mx0 = fmaxf(mx0, fmaxf(sv[nt][0], sv[nt][2]));
+          mx1 = fmaxf(mx1, fmaxf(sv[nt][1], sv[nt][3]));
+        }
+#pragma unroll
+        for (int off = 4; off < 32; off <<= 1) {
+          mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+          mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+        }
+        // Lazy rescale: the max moves only when it grows by more than the
+        // threshold (p stays below 2^threshold, well inside f16 and bf16).
+        const bool need0 = mx0 > m0 + kRescaleThreshold, need1 = mx1 > m1 + kRescaleThreshold;
+        float al0 = 1.f, al1 = 1.f;
+        if (need0) {
+          al0 = exp2f(m0 - mx0);
+          m0 = mx0;
+          l0 *= al0;
+        }
+        if (need1) {
+          al1 = exp2f(m1 - mx1);
+          m1 = mx1;
+          l1 *= al1;
+        }
+        if (__any_sync(0xffffffffu, need0 || need1)) {
+#pragma unroll
+          for (int mt = 0; mt < 8; ++mt) {
+            acc[mt][0] *= al0;
+            acc[mt][2] *= al0;
+            acc[mt][1] *= al1;
+            acc[mt][3] *= al1;
+          }
+        }
+        auto to16 = [](float x) -> uint16_t {
+          if constexpr (kF8) return __half_as_ushort(__float2half_rn(x));
+          else return __bfloat16_as_ushort(__float2bfloat16_rn(x));
+        };
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          const float p00 = v0 ? exp2f(sv[nt][0] - m0) : 0.f, p10 = v0 ? exp2f(sv[nt][2] - m0) : 0.f;
+          const float p01 = v1 ? exp2f(sv[nt][1] - m1) : 0.f, p11 = v1 ? exp2f(sv[nt][3] - m1) : 0.f;
+          l0 += p00 + p10;
+          l1 += p01 + p11;
+          if (v0) {
+            pw[(2 * kq) * kPS + 16 * nt + qr] = to16(p00);
+            pw[(2 * kq) * kPS + 16 * nt + qr + 8] = to16(p10);
+          }
+          if (v1) {
+            pw[(2 * kq + 1) * kPS + 16 * nt + qr] = to16(p01);
+            pw[(2 * kq + 1) * kPS + 16 * nt + qr + 8] = to16(p11);
+          }
+        }
+        __syncwarp();
+        // P^T B fragments: b0 = p of head qr at tokens 2kq, 2kq + 1 of the
+        // tile; b1 at + 8.
+        uint32_t pb[NT][2];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          pb[nt][0] = pb[nt][1] = 0u;
+          if (qr < G) {
+            pb[nt][0] = *reinterpret_cast<const uint32_t*>(pw + qr * kPS + 16 * nt + 2 * kq);
+            pb[nt][1] = *reinterpret_cast<const uint32_t*>(pw + qr * kPS + 16 * nt + 2 * kq + 8);
+          }
+        }
+        __syncwarp();
+        // ---- PV -------------------------------------------------------------
+        // In a partial tile, tokens outside [lo, hi) are not this piece's
+        // (stale, unwritten or other pages' rows): their V entries are zeroed
+        // in the A fragments, since p = 0 would not clear a non-finite value.
+        auto pv_tile = [&](int nt, auto masked_tag) {
+          constexpr bool kMasked = decltype(masked_tag)::value;
+          uint32_t mlo = 0xffffffffu, mhi = 0xffffffffu;
+          if constexpr (kMasked) {
+            const int lo = lo_t[nt], hi = hi_t[nt];
+            auto in = [&](int t) { return t >= lo && t < hi; };
+            mlo = (in(2 * kq) ? 0x0000ffffu : 0u) | (in(2 * kq + 1) ? 0xffff0000u : 0u);
+            mhi = (in(2 * kq + 8) ? 0x0000ffffu : 0u) | (in(2 * kq + 9) ? 0xffff0000u : 0u);
+          }
+          if constexpr (kF8) {
+#pragma unroll
+            for (int pp = 0; pp < 4; ++pp) {
+              uint32_t w[4];
+              ldsm_x4_trans(v_addr(nt, pp), w);
+              // w[j] = codes (token 2kq: dims 2qr, 2qr + 1 | token 2kq + 1:
+              // same dims) of matrix j = (chunk 2pp | 2pp + 1) x (tokens 0-7 | 8-15).
+              uint32_t fe[4], fo[4];
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                const uint32_t x = __byte_perm(w[j], 0u, 0x3120);  // (t0 even, t1 even, t0 odd, t1 odd)
+                fe[j] = lo_f16x2(x);
+                fo[j] = hi_f16x2(x);
+                if constexpr (kMasked) {
+                  fe[j] &= j < 2 ? mlo : mhi;
+                  fo[j] &= j < 2 ? mlo : mhi;
+                }
+              }
+              mma16816<true>(acc[2 * pp], fe, pb[nt][0], pb[nt][1]);
+              mma16816<true>(acc[2 * pp + 1], fo, pb[nt][0], pb[nt][1]);
+            }
+          } else {
+#pragma unroll
+            for (int mt = 0; mt < 8; ++mt) {
+              uint32_t f[4];
+              ldsm_x4_trans(v_addr(nt, mt), f);
+              if constexpr (kMasked) {
+                f[0] &= mlo;
+                f[1] &= mlo;
+                f[2] &= mhi;
+                f[3] &= mhi;
+              }
+              mma16816<false>(acc[mt], f, pb[nt][0], pb[nt][1]);
+            }
+          }
+        };
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          if (lo_t[nt] == 0 && hi_t[nt] == 16)
+            pv_tile(nt, std::false_type{});
+          else if (hi_t[nt] > lo_t[nt])
+            pv_tile(nt, std::true_type{});
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[slot_i]);
+        j0 = jn;
+        ++s;
+      }
+
+      // ---- finish the piece -------------------------------------------------
+#pragma unroll
+      for (int off = 4; off < 32; off <<= 1) {
+        l0 += __shfl_xor_sync(0xffffffffu, l0, off);
+        l1 += __shfl_xor_sync(0xffffffffu, l1, off);
+      }
+      // Output dims of accumulator (mt, e): bf16 rows: 16 mt + qr (+ 8 for
+      // e >= 2); FP8 rows: 32 (mt / 2) + 2 qr + (mt & 1) (+ 16 for e >= 2).
+#pragma unroll
+      for (int hs = 0; hs < 2; ++hs) {
+        if (!(hs == 0 ? v0 : v1)) continue;
+        const int h = g * G + 2 * kq + hs;
+        const float lsum = hs == 0 ? l0 : l1, mh = hs == 0 ? m0 : m1;
+        const float vs = kF8 ? a.v_scale : 1.f;
+        if (whole) {
+          const float inv = lsum > 0.f ? vs / lsum : 0.f;
+          IO* orow = obase + ((int64_t)r * a.hq + h) * kHeadDim;
+          if constexpr (kF8) {
+#pragma unroll
+            for (int pp = 0; pp < 4; ++pp) {
+#pragma unroll
+              for (int up = 0; up < 2; ++up) {
+                const uint32_t w = pack_bf16x2(acc[2 * pp][hs + 2 * up] * inv, acc[2 * pp + 1][hs + 2 * up] * inv);
+                *reinterpret_cast<uint32_t*>(orow + 32 * pp + 16 * up + 2 * qr) = w;
+              }
+            }
+          } else {
+#pragma unroll
+            for (int mt = 0; mt < 8; ++mt) {
+              orow[16 * mt + qr] = __float2bfloat16_rn(acc[mt][hs] * inv);
+              orow[16 * mt + qr + 8] = __float2bfloat16_rn(acc[mt][hs + 2] * inv);
+            }
+          }
+        } else {
+          const int64_t id = static_cast<int64_t>(blockIdx.x) + r;
+          float* op = a.ws_o + (id * a.hq + h) * kHeadDim;
+          if constexpr (kF8) {
+#pragma unroll
+            for (int pp = 0; pp < 4; ++pp)
+#pragma unroll
+              for (int up = 0; up < 2; ++up)
+                *reinterpret_cast<float2*>(op + 32 * pp + 16 * up + 2 * qr) =
+                    make_float2(acc[2 * pp][hs + 2 * up] * vs, acc[2 * pp + 1][hs + 2 * up] * vs);
+          } else {
+#pragma unroll
+            for (int mt = 0; mt < 8; ++mt) {
+              op[16 * mt + qr] = acc[mt][hs];
+              op[16 * mt + qr + 8] = acc[mt][hs + 2];
+            }
+          }
+          if (qr == 0) a.ws_ml[id * a.hq + h] = make_float2(mh, lsum);
+        }
+      }
+    }
+  } else {
   // ============================= consumers ==================================
   // Scores use the token-group lane map (tl, d) = (lane / D, lane % D); the
   // PV product uses (half, c) = (lane / 16, lane % 16): lane c owns dims
@@ -493,7 +1098,7 @@ __global__ void __launch_bounds__(32 * 9, 1) decode_split_kernel(const DecodeArg
       }
       const int ntok = static_cast<int>(min((int64_t)T, jb - j0));
       const uint8_t* kst = ring + slot_i * L.stage_bytes;
-      const uint8_t* vst = kst + T * a.row_bytes;
+      const uint8_t* vst = kst + T * RS;
 
 #pragma unroll
       for (int sub = 0; sub < T; sub += SUB) {
@@ -506,11 +1111,11 @@ __global__ void __launch_bounds__(32 * 9, 1) decode_split_kernel(const DecodeArg
           float2 acc[G];
           float2 kw[UPL][4];
           if constexpr (kWideFp8) {
-            load16_e4m3(kst + t * a.row_bytes + g * kHeadDim + 16 * d, kw[0], kw[UPL - 1]);
+            load16_e4m3(kst + t * RS + g * kHeadDim + 16 * d, kw[0], kw[UPL - 1]);
           } else {
 #pragma unroll
             for (int m = 0; m < UPL; ++m)
-              load8<E>(reinterpret_cast<const E*>(kst + t * a.row_bytes + (g * kHeadDim + unit_dim(m)) * ESZ),
+              load8<E>(reinterpret_cast<const E*>(kst + t * RS + (g * kHeadDim + unit_dim(m)) * ESZ),
                        kw[m]);
           }
 #pragma unroll
@@ -575,7 +1180,7 @@ __global__ void __launch_bounds__(32 * 9, 1) decode_split_kernel(const DecodeArg
           const int tt = 2 * i + half;
           if (sub + tt < ntok) {
             float2 v2[4];
-            load8<E>(reinterpret_cast<const E*>(vst + (sub + tt) * a.row_bytes + (g * kHeadDim + 8 * c) * ESZ), v2);
+            load8<E>(reinterpret_cast<const E*>(vst + (sub + tt) * RS + (g * kHeadDim + 8 * c) * ESZ), v2);
             float p[G];
             load_p<G>(pw + tt * G, p);
 #pragma unroll
@@ -640,6 +1245,7 @@ __global__ void __launch_bounds__(32 * 9, 1) decode_split_kernel(const DecodeArg
         if (c == 0) a.ws_ml[id * a.hq + h] = make_float2(mh[hh], lsum[hh]);
       }
     }
+  }
   }
 }
 
@@ -713,15 +1319,48 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(
   }
 }
 
-template <typename E, int G>
-cudaError_t launch_decode_t(const DecodeArgs& a, int grid, cudaStream_t s, const CascadeView* cv) {
+// Tensor map of one pool plane for page-box stages (see tma_page_box): slot
+// is the second dimension, so a box of 16 slots lands as 16 consecutive
+// 128-byte rows per head (and half row), which the 128B swizzle spreads over
+// all banks for the consumers' ldmatrix reads.
+bool make_page_map(CUtensorMap* map, const uint8_t* base, int64_t num_slots, int64_t slot_stride, int hkv,
+                   bool fp8) {
+  auto fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(tensor_map_encode_fn());
+  if (fn == nullptr || num_slots < 16) return false;
+  void* gaddr = const_cast<uint8_t*>(base);
+  if (fp8) {
+    cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(num_slots), static_cast<cuuint64_t>(hkv)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(slot_stride), 128};
+    cuuint32_t box[3] = {128, 16, static_cast<cuuint32_t>(hkv)};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, gaddr, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  }
+  cuuint64_t dims[4] = {64, static_cast<cuuint64_t>(num_slots), 2, static_cast<cuuint64_t>(hkv)};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(slot_stride), 128, 256};
+  cuuint32_t box[4] = {64, 16, 2, static_cast<cuuint32_t>(hkv)};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, gaddr, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <typename E, int G, bool kPaged>
+cudaError_t launch_split_t(const DecodeArgs& a, int grid, cudaStream_t s, const CascadeView* cv,
+                           const CUtensorMap& kmap, const CUtensorMap& vmap) {
   constexpr int T = DecodeTraits<E>::kTokensPerStage;
-  const DecodeSmem L = decode_smem_layout(a.batch, a.hkv, a.row_bytes, T, G);
+  using LT = DecodeLayoutTraits<E>;
+  constexpr int kPsm = LT::template psm_per_warp<G>();
+  constexpr int kPad = kPaged ? 0 : LT::kRowPad;
+  constexpr int kSlack = kPaged ? 1024 : 0;  // in-kernel 1024-byte alignment of the stages
+  const DecodeSmem L = decode_smem_layout(a.batch, a.hkv, a.row_bytes + kPad, T, kPsm);
   // The limit is raised once to the largest layout any batch can need.
   static int smem_state[kMaxDevicesHost] = {};
-  const int max_bytes = decode_smem_layout(kMaxBatch, 8, 8 * kHeadDim * static_cast<int>(sizeof(E)), T, G).total;
-  if (L.total > max_bytes) return cudaErrorInvalidValue;
-  cudaError_t e = ensure_smem_limit(decode_split_kernel<E, G>, max_bytes, smem_state);
+  const int max_bytes =
+      decode_smem_layout(kMaxBatch, 8, 8 * kHeadDim * static_cast<int>(sizeof(E)) + kPad, T, kPsm).total + kSlack;
+  if (L.total + kSlack > max_bytes) return cudaErrorInvalidValue;
+  cudaError_t e = ensure_smem_limit(decode_split_kernel<E, G, kPaged>, max_bytes, smem_state);
   if (e != cudaSuccess) return e;
   // Both kernels use programmatic dependent launch: the split kernel is
   // scheduled and sets up its barriers while the preceding kernel finishes,
@@ -734,11 +1373,11 @@ cudaError_t launch_decode_t(const DecodeArgs& a, int grid, cudaStream_t s, const
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(32 * (1 + a.hkv));
-  cfg.dynamicSmemBytes = L.total;
+  cfg.dynamicSmemBytes = L.total + kSlack;
   cfg.stream = s;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, decode_split_kernel<E, G>, a);
+  e = cudaLaunchKernelEx(&cfg, decode_split_kernel<E, G, kPaged>, a, kmap, vmap);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t ccfg = cfg;
   ccfg.gridDim = dim3(a.batch, (a.hq + 3) / 4);
@@ -749,6 +1388,23 @@ cudaError_t launch_decode_t(const DecodeArgs& a, int grid, cudaStream_t s, const
                             (const int64_t*)a.ws_per, (const float2*)a.ws_ml, (const float*)a.ws_o,
                             a.hq, a.out, cv ? cv->pre_ml : nullptr, cv ? cv->pre_o : nullptr,
                             cv ? cv->nsplit : 0);
+}
+
+// Page sizes that are multiples of 16 take page-box stages (bf16 and FP8
+// pools); every other pool streams token rows.
+template <typename E, int G>
+cudaError_t launch_decode_t(const DecodeArgs& a, int grid, cudaStream_t s, const CascadeView* cv) {
+  if constexpr (DecodeLayoutTraits<E>::kMma) {
+    if (a.page_size % 16 == 0) {
+      CUtensorMap km, vm;
+      if (make_page_map(&km, a.kbase, a.num_slots, a.slot_stride_bytes, a.hkv, sizeof(E) == 1) &&
+          make_page_map(&vm, a.vbase, a.num_slots, a.slot_stride_bytes, a.hkv, sizeof(E) == 1))
+        return launch_split_t<E, G, true>(a, grid, s, cv, km, vm);
+    }
+  }
+  CUtensorMap none;
+  memset(&none, 0, sizeof(none));
+  return launch_split_t<E, G, false>(a, grid, s, cv, none, none);
 }
 
 }  // namespace

@@ -28,6 +28,9 @@ inline cudaError_t ensure_smem_limit(Kernel kernel, int bytes, int* state) {
   return e;
 }
 
+// Driver entry point of cuTensorMapEncodeTiled (null when unavailable).
+void* tensor_map_encode_fn();
+
 struct PoolView {
   const uint8_t* k;  // layer base (bytes)
   const uint8_t* v;
