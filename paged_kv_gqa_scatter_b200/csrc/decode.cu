@@ -12,29 +12,32 @@
 //    may hold the tail of one request, whole requests and the head of another;
 //    each (request, CTA) intersection is a "piece".  Equal ranges balance the
 //    HBM traffic across SMs exactly, whatever the length mix.
-//  * Warp 0 is the producer: for each stage of 16 tokens it translates the
-//    tokens' slots through the page table and issues one 1-D bulk copy
-//    (cp.async.bulk, the TMA's non-tensor form) per token and plane.  A token
-//    row holds all KV heads of the slot (2 KB for 8 heads x 128 x bf16), so
-//    every copy is a long contiguous read.  Stages live in a 3-deep ring of
-//    shared memory guarded by full/empty mbarriers.
-//  * Warps 1..Hkv are consumers, one per KV head.  Lane = (half, c): c picks
-//    8 consecutive dims, half picks even/odd tokens.  Scores for 8 tokens x G
-//    heads are reduced across the 16 lanes of a half with a transposing
-//    butterfly (each step halves the values a lane keeps), so the reduction
-//    costs about one shuffle per (token, head) instead of four.  Softmax runs
-//    in the log2 domain with exp2 and a lazily moved running max (the
-//    accumulators are rescaled only when the max grows by more than 2^8).
-//    PV accumulates with packed f32x2 FMAs.
+//  * Warp 0 is the producer; stages live in a 3-deep shared-memory ring
+//    guarded by full/empty mbarriers.  Pools whose page size is a multiple of
+//    16 load a stage as page boxes: one tensor copy per plane for every 16
+//    table columns (aligned to 16, so inside one page), 16 consecutive slots
+//    of all KV heads (32 KB at Hkv 8, bf16), 128B-swizzled.  Other page sizes
+//    translate every token's slot and issue one 1-D bulk copy per token row
+//    and plane into rows padded by 16 bytes.  Measured on B200, bulk copies
+//    top out near 3 G copies per second, so large copies are what reach the
+//    HBM bandwidth.
+//  * Warps 1..Hkv are consumers, one per KV head.  bf16 and FP8 pools use
+//    tensor cores (mma.sync m16n8k16, fp32 accumulate) with the GQA group as
+//    the N dimension: S^T = K Q^T over 16-token tiles, then O^T += V^T P^T,
+//    fragments read with ldmatrix (transposed for V).  FP8 codes widen
+//    exactly to f16.  Softmax runs in the log2 domain with exp2 and a lazily
+//    moved running max (the accumulators are rescaled only when the max grows
+//    by more than 2^8); p passes to the PV fragments through a small per-warp
+//    buffer.  fp32 pools (the check build) keep CUDA-core dot products with a
+//    transposing butterfly reduction and packed f32x2 FMAs.
 //  * A piece that covers a whole request writes the final output; other
 //    pieces write an un-normalised fp32 partial plus (max, sum) to the
 //    workspace and decode_combine_kernel merges them.
 //  * Cascade suffix pass (cascade.cu): each request starts at its own table
 //    column, every piece writes a partial, and the combine kernel also merges
 //    the shared-prefix partials.
-//  * FP8 (E4M3) pools: 32 tokens per stage (1 KB rows); codes widen exactly to
-//    half and then float; the K scale is folded into the softmax scale and
-//    the V scale into the output.
+//  * FP8 (E4M3) pools: 32 tokens per stage; the K scale is folded into the
+//    softmax scale and the V scale into the output.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>

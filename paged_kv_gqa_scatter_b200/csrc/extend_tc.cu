@@ -837,8 +837,6 @@ cudaError_t launch_for_pool(const PoolView& pool, int G, const CUtensorMap& qm, 
 
 }  // namespace
 
-void* tensor_map_encode_fn() { return reinterpret_cast<void*>(encode_fn()); }
-
 cudaError_t launch_extend_tc(const PoolView& pool, const TableView& t, const void* q, int32_t num_q_heads,
                              const int32_t* table_idx, const int32_t* prefix_lens, const int32_t* extend_lens,
                              const int32_t* q_offsets, int32_t batch, int64_t total_q, int32_t max_extend,
