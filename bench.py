@@ -423,6 +423,8 @@ def run_decode(args, world, rank, local, name):
     if name == "decode-qwen3-8b":
         free, _ = torch.cuda.mem_get_info()
         wl, pool_note = qwen3_8b_workload(args, free)
+        if args.kv_dtype == "fp8":
+            wl = W.with_fp8_pool(wl)
         layers = list(range(wl.pool.num_layers))
     else:
         nl = 28 if args.pool_layers is None else args.pool_layers
@@ -1102,7 +1104,7 @@ def main():
     ap.add_argument("--page-size", type=int, default=None,
                     help="page size of decode-qwen3-8b (16 as stated; 64 is TRT-LLM's size)")
     ap.add_argument("--kv-dtype", choices=["bf16", "fp8"], default="bf16",
-                    help="pool element type of decode-qwen3-0.6b (fp8: scaled E4M3 codes, bf16 q/out)")
+                    help="pool element type of the decode workloads (fp8: scaled E4M3 codes, bf16 q/out)")
     ap.add_argument("--radix-decode", choices=["cascade", "plain"], default="cascade",
                     help="decode call of the radix-prefix workload's step")
     args = ap.parse_args()

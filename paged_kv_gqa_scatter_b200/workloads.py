@@ -746,11 +746,16 @@ def with_fp8_pool(wl, k_scale: float = 0.05, v_scale: float = 0.09, seed: Option
     the stored codes of the new rows depend on float32 rounding of
     x * (1 / scale)."""
     rng = np.random.Generator(np.random.PCG64(seed_for(8) if seed is None else seed))
-    if wl.pool.dtype != BF16 or isinstance(wl.k_planes, TiledPlane):
-        raise ValueError("needs a bf16 workload with dict planes")
+    if wl.pool.dtype != BF16:
+        raise ValueError("needs a bf16 workload")
     spec = dataclasses.replace(wl.pool, dtype=F8, k_scale=float(np.float32(k_scale)),
                                v_scale=float(np.float32(v_scale)))
-    shape = (spec.num_slots, spec.num_kv_heads, spec.head_dim)
-    kp = {l: draw_e4m3_codes(rng, shape) for l in wl.k_planes}
-    vp = {l: draw_e4m3_codes(rng, shape) for l in wl.v_planes}
+    if isinstance(wl.k_planes, TiledPlane):
+        # Tiled pools (decode-qwen3-8b): a code block of the same size, tiled the same way.
+        kp = TiledPlane(draw_e4m3_codes(rng, wl.k_planes.block.shape), spec.num_layers, spec.num_slots)
+        vp = TiledPlane(draw_e4m3_codes(rng, wl.v_planes.block.shape), spec.num_layers, spec.num_slots)
+    else:
+        shape = (spec.num_slots, spec.num_kv_heads, spec.head_dim)
+        kp = {l: draw_e4m3_codes(rng, shape) for l in wl.k_planes}
+        vp = {l: draw_e4m3_codes(rng, shape) for l in wl.v_planes}
     return dataclasses.replace(wl, name=wl.name + "-fp8", pool=spec, k_planes=kp, v_planes=vp)

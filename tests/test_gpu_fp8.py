@@ -29,6 +29,16 @@ pytestmark = pytest.mark.gpu
 D = W.HEAD_DIM
 
 
+def scale_check(got: np.ndarray, exp: np.ndarray, what: str, frac: float = 1e-2):
+    """Decode outputs over E4M3 pools average many random-sign values, so they
+    are small (about 0.01-0.1) next to the 1e-2 absolute bound; also require
+    the error to stay within `frac` of the largest output magnitude.  The
+    kernel's own error (p rounded to f16 before PV) is far below that."""
+    err = float(np.abs(got - exp).max())
+    bound = frac * float(np.abs(exp).max())
+    assert err <= bound, f"{what}: max error {err:.3e} above {frac} x max |ref| = {bound:.3e}"
+
+
 def _codes(t: torch.Tensor) -> np.ndarray:
     return t.view(torch.uint8).cpu().numpy()
 
@@ -103,6 +113,7 @@ def test_fp8_decode_matches_oracle(maker, hq):
     kp, vp = _oracle_store(wl)
     exp = _oracle_decode(wl, kp, vp)
     tol_check(from_dev(d.out), exp, W.BF16, f"fp8 decode {maker} hq={hq}")
+    scale_check(from_dev(d.out), exp, f"fp8 decode {maker} hq={hq}")
 
 
 def test_fp8_decode_qwen3_06b_full():
@@ -118,6 +129,48 @@ def test_fp8_decode_qwen3_06b_full():
     req = sorted(rng.choice(wl.batch, 12, replace=False).tolist())
     exp = _oracle_decode(wl, kp, vp, requests=req)
     tol_check(from_dev(d.out)[req], exp[req], W.BF16, "fp8 decode-qwen3-0.6b")
+    scale_check(from_dev(d.out)[req], exp[req], "fp8 decode-qwen3-0.6b")
+
+
+class _DequantPlanes:
+    """Code planes (dict or tiled) read as float64 values code * scale, slot by
+    slot, so a tiled pool never has to be decoded whole."""
+
+    def __init__(self, planes, scale):
+        self.planes, self.scale = planes, float(np.float32(scale))
+
+    def __getitem__(self, layer):
+        view = self.planes[layer]
+        scale = self.scale
+
+        class _Layer:
+            def __getitem__(self, slots):
+                return oracle.e4m3_decode(view[slots]) * scale
+
+        return _Layer()
+
+
+def test_fp8_decode_qwen3_8b_sampled():
+    """The headline batch (256 requests, 1k-32k, page size 16, so decode loads
+    page boxes) over an E4M3 copy of one layer of its pool: 16 sampled
+    requests, the longest and shortest included."""
+    from gpu_helpers import host_planes_copy
+    wl = W.with_fp8_pool(W.decode_qwen3_8b(num_layers=1))
+    d = DeviceDecode(wl)
+    d.run()
+    torch.cuda.synchronize()
+    assert int(d.err.item()) == 0
+    kp, vp = host_planes_copy(wl.k_planes), host_planes_copy(wl.v_planes)
+    oracle.store_kv_fp8(kp, vp, wl.layer, wl.k_new, wl.v_new, wl.out_loc, wl.pool.num_kv_heads, D,
+                        wl.pool.k_scale, wl.pool.v_scale)
+    lens = wl.seq_lens
+    req = sorted(set([int(np.argmax(lens)), int(np.argmin(lens))] +
+                     np.random.default_rng(5).choice(wl.batch, 14, replace=False).tolist()))
+    exp = oracle.decode_attn(wl.q, _DequantPlanes(kp, wl.pool.k_scale), _DequantPlanes(vp, wl.pool.v_scale),
+                             wl.layer, wl.page_table, wl.table_idx, wl.seq_lens, wl.pool.page_size, wl.scale,
+                             requests=req)
+    tol_check(from_dev(d.out)[req], exp[req], W.BF16, "fp8 decode-qwen3-8b")
+    scale_check(from_dev(d.out)[req], exp[req], "fp8 decode-qwen3-8b")
 
 
 def test_fp8_rope_store():
