@@ -1287,13 +1287,14 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(
   const int64_t per = *per_p;
   const int64_t k_lo = c1 > c0 ? c0 / per : 0, k_hi = c1 > c0 ? (c1 - 1) / per : -1;
   if (!cascade && k_lo == k_hi) return;  // written by its only piece
-  // Online merge: the loads of consecutive pieces are independent, so the
-  // unrolled loops keep several in flight.
+  // Online merge.  Partials are taken eight at a time, all of a batch's
+  // loads ((max, sum) pairs and output slices, independent of each other)
+  // issued before any merge, so a batch costs about one memory round trip.
+  // Cascade mode merges the nsplit shared-prefix partials first.
   float M = -INFINITY, den = 0.f;
   float4 acc = make_float4(0, 0, 0, 0);
-  auto merge = [&](float2 st, const float* src) {
-    if (!(st.y > 0.f)) return;  // empty partial
-    const float4 x = *reinterpret_cast<const float4*>(src + 4 * lane);
+  auto merge = [&](float2 st, float4 x) {
+    if (!(st.y > 0.f)) return;  // empty partial (its output slice is not read)
     const float Mn = fmaxf(M, st.x);
     const float wa = exp2f(M - Mn), wb = exp2f(st.x - Mn);
     den = den * wa + wb * st.y;
@@ -1304,13 +1305,27 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(
     M = Mn;
   };
   const int64_t B = gridDim.x;
-#pragma unroll 4
-  for (int sp = 0; sp < nsplit; ++sp) {
-    const int64_t id = (sp * B + r) * hq + h;
-    merge(pre_ml[id], pre_o + id * kHeadDim);
+  const int64_t npre = cascade ? nsplit : 0;
+  const int64_t total = npre + (k_hi - k_lo + 1);
+  constexpr int kBatch = 8;
+  for (int64_t b0 = 0; b0 < total; b0 += kBatch) {
+    float2 st[kBatch];
+    float4 x[kBatch];
+#pragma unroll
+    for (int i = 0; i < kBatch; ++i) {
+      const int64_t t = b0 + i;
+      st[i] = make_float2(-INFINITY, 0.f);
+      x[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (t < total) {
+        const bool pre = t < npre;
+        const int64_t id = pre ? (t * B + r) * hq + h : (k_lo + (t - npre) + r) * hq + h;
+        st[i] = (pre ? pre_ml : ml)[id];
+        x[i] = *reinterpret_cast<const float4*>((pre ? pre_o : o) + id * kHeadDim + 4 * lane);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < kBatch; ++i) merge(st[i], x[i]);
   }
-#pragma unroll 4
-  for (int64_t k = k_lo; k <= k_hi; ++k) merge(ml[(k + r) * hq + h], o + ((k + r) * hq + h) * kHeadDim);
   const float inv = den > 0.f ? 1.f / den : 0.f;
   if constexpr (sizeof(E) == 2) {
     uint2 w;

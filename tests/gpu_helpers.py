@@ -168,3 +168,18 @@ def oracle_extend(wl: W.ExtendWorkload, rows=None, planes=None):
     out = oracle.extend_attn(wl.q, kp, vp, wl.layer, wl.page_table, wl.table_idx, wl.prefix_lens,
                              wl.extend_lens, wl.q_offsets, wl.pool.page_size, wl.scale, rows=rows)
     return out, (kp, vp)
+
+
+def referenced_slots(wl) -> np.ndarray:
+    """Pool slots that some request's context reads (the stored token included)."""
+    used = [oracle.slots_of(wl.page_table, int(wl.table_idx[r]), int(wl.seq_lens[r]), wl.pool.page_size)
+            for r in range(wl.batch)]
+    return np.unique(np.concatenate(used))
+
+
+def poison_unreferenced(planes, layer, keep, value):
+    """Set every slot of `layer` outside `keep` to `value` (a NaN pattern)."""
+    a = planes[layer]
+    mask = np.ones(a.shape[0], dtype=bool)
+    mask[keep] = False
+    a[mask] = value

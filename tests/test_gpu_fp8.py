@@ -173,6 +173,27 @@ def test_fp8_decode_qwen3_8b_sampled():
     scale_check(from_dev(d.out)[req], exp[req], "fp8 decode-qwen3-8b")
 
 
+def test_fp8_decode_nan_codes_in_unreferenced_slots():
+    """Every slot no context reads holds the E4M3 NaN code 0x7F; page boxes load
+    the tails of last pages and the rows before a CTA's first token, which must
+    be masked out (p = 0 does not clear NaN)."""
+    from gpu_helpers import poison_unreferenced, referenced_slots
+    wl = W.with_fp8_pool(W.decode_paged_small(page_size=16, seq_lens=(1, 15, 17, 33, 300, 1029, 47),
+                                              seed=1600), seed=7)
+    keep = referenced_slots(wl)
+    for planes in (wl.k_planes, wl.v_planes):
+        poison_unreferenced(planes, 0, keep, np.uint8(0x7F))
+    d = DeviceDecode(wl)
+    d.run()
+    torch.cuda.synchronize()
+    assert int(d.err.item()) == 0
+    assert torch.isfinite(d.out.float()).all(), "a masked NaN row reached the output"
+    kp, vp = _oracle_store(wl)
+    exp = _oracle_decode(wl, kp, vp)
+    tol_check(from_dev(d.out), exp, W.BF16, "fp8 decode, NaN codes in unreferenced slots")
+    scale_check(from_dev(d.out), exp, "fp8 decode, NaN codes in unreferenced slots")
+
+
 def test_fp8_rope_store():
     wl = W.rope_store_step(W.BF16, seed=31)
     hq, hkv = wl.num_q_heads, wl.pool.num_kv_heads

@@ -14,6 +14,7 @@ import torch
 
 import oracle
 from gpu_helpers import (DeviceDecode, DeviceExtend, device_pool, from_dev, host_planes_copy, i32,
+                         poison_unreferenced, referenced_slots,
                          oracle_decode, oracle_extend, to_dev, tol_check)
 from paged_kv_gqa_scatter_b200 import api
 from paged_kv_gqa_scatter_b200 import workloads as W
@@ -146,6 +147,42 @@ def test_decode_group_sizes(dtype, hq, hkv):
     d.run()
     exp, _ = oracle_decode(wl)
     tol_check(from_dev(d.out), exp, dtype, f"decode hq={hq} hkv={hkv}")
+
+
+@pytest.mark.parametrize("dtype", DTYPES)
+@pytest.mark.parametrize("hq,hkv", [(4, 1), (16, 2), (32, 4), (64, 8)])
+def test_decode_paged_group_sizes(dtype, hq, hkv):
+    """page_size 16 (page-box stages for bf16) with 1, 2, 4 and 8 KV heads:
+    boxes of 4 to 32 KB per plane."""
+    wl = W.decode_paged_small(dtype=dtype, num_q_heads=hq, num_kv_heads=hkv, seed=1400 + hq + hkv)
+    d = DeviceDecode(wl)
+    d.run()
+    exp, _ = oracle_decode(wl)
+    tol_check(from_dev(d.out), exp, dtype, f"decode P=16 hq={hq} hkv={hkv}")
+    assert _err(d.err) == 0
+
+
+@pytest.mark.parametrize("dtype", DTYPES)
+@pytest.mark.parametrize("page_size,hq,hkv", [(16, 32, 8), (16, 8, 2), (64, 16, 8), (1, 16, 8)])
+def test_decode_nan_in_unreferenced_slots(dtype, page_size, hq, hkv):
+    """Every slot no context reads holds NaN.  Page boxes load whole 16-slot
+    groups, so the tails of last pages and the rows before a CTA's first token
+    reach shared memory; they must be masked out of the scores and the PV
+    product (p = 0 does not clear NaN)."""
+    wl = W.decode_paged_small(dtype=dtype, page_size=page_size, num_q_heads=hq, num_kv_heads=hkv,
+                              seq_lens=(1, 15, 17, 33, 300, 1029, 47), seed=1500 + page_size)
+    nan = np.uint16(0x7FC0) if dtype == W.BF16 else np.float32("nan")
+    keep = referenced_slots(wl)
+    assert keep.shape[0] < wl.pool.num_slots
+    for planes in (wl.k_planes, wl.v_planes):
+        poison_unreferenced(planes, 0, keep, nan)
+    d = DeviceDecode(wl)
+    d.run()
+    torch.cuda.synchronize()
+    assert torch.isfinite(d.out.float()).all(), "a masked NaN row reached the output"
+    exp, _ = oracle_decode(wl)
+    tol_check(from_dev(d.out), exp, dtype, f"decode with NaN in unreferenced slots P={page_size}")
+    assert _err(d.err) == 0
 
 
 def test_decode_one_token_returns_v_exactly():
