@@ -12,16 +12,17 @@
 //    may hold the tail of one request, whole requests and the head of another;
 //    each (request, CTA) intersection is a "piece".  Equal ranges balance the
 //    HBM traffic across SMs exactly, whatever the length mix.
-//  * Warp 0 is the producer; stages live in a 3-deep shared-memory ring
-//    guarded by full/empty mbarriers.  Pools whose page size is a multiple of
+//  * Warps 0..3 are producers (one for fp32 pools), each copying one plane
+//    (K or V) of every other token or page group and arming the stage's full
+//    barrier for its own bytes: one warp issuing bulk copies tops out near
+//    3 G copies/s.  Stages live in a 3-deep shared-memory ring guarded by
+//    full/empty mbarriers.  Pools whose page size is a multiple of
 //    16 load a stage as page boxes: one tensor copy per plane for every 16
 //    table columns (aligned to 16, so inside one page), 16 consecutive slots
 //    of all KV heads (32 KB at Hkv 8, bf16), 128B-swizzled.  Other page sizes
 //    translate every token's slot and issue one 1-D bulk copy per token row
-//    and plane into rows padded by 16 bytes.  Measured on B200, bulk copies
-//    top out near 3 G copies per second, so large copies are what reach the
-//    HBM bandwidth.
-//  * Warps 1..Hkv are consumers, one per KV head.  bf16 and FP8 pools use
+//    and plane into rows padded by 16 bytes.
+//  * The next Hkv warps are consumers, one per KV head.  bf16 and FP8 pools use
 //    tensor cores (mma.sync m16n8k16, fp32 accumulate) with the GQA group as
 //    the N dimension: S^T = K Q^T over 16-token tiles, then O^T += V^T P^T,
 //    fragments read with ldmatrix (transposed for V).  FP8 codes widen
