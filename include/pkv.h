@@ -284,7 +284,8 @@ int pkv_gather_kv(const pkv_pool* pool, int32_t layer, const pkv_page_table* tab
  * out: device [batch][num_q_heads][head_dim] contiguous, q's dtype
  *   (fp32 accumulation, rounded to nearest-even on store).  bf16 and FP8
  *   pools compute on tensor cores: the softmax weights enter the PV product
- *   rounded to bf16 (bf16 pools) or f16 (FP8 pools); fp32 pools stay fp32.
+ *   as two bf16 terms (bf16 pools, about 16 significant bits) or rounded to
+ *   f16 (FP8 pools); fp32 pools stay fp32.
  * table_idx, seq_lens: device int32 [batch].
  * scale: softmax scale (the pages do not state it; 1/sqrt(head_dim) is the
  *   usual choice).

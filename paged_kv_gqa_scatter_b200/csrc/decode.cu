@@ -142,9 +142,12 @@ struct DecodeLayoutTraits {
   // copies/s (measured on B200: 3.1 TB/s at 1 KB rows); four warps, each
   // copying one plane for every other token, reach the HBM bandwidth.
   static constexpr int kProd = kMma ? 4 : 1;
+  // bf16 pools pass p to the PV product as two bf16 terms, p = hi + lo (to
+  // about 2^-17 relative), in two buffers; f16 (FP8 pools) keeps 11 bits.
+  static constexpr bool kSplitP = kMma && sizeof(E) == 2;
   template <int G>
   static constexpr int psm_per_warp() {
-    return kMma ? 8 * kPStride * 2 : 4 * DecodeTraits<E>::kTokensPerStage * G;
+    return kMma ? 8 * kPStride * 2 * (kSplitP ? 2 : 1) : 4 * DecodeTraits<E>::kTokensPerStage * G;
   }
 };
 
@@ -693,8 +696,10 @@ __global__ void __launch_bounds__(32 * 12, 1) decode_split_kernel(const DecodeAr
     // so its softmax state (max, sum) covers exactly the heads whose output it
     // accumulates.  P passes from the score layout to the PV B fragment
     // through the warp's p buffer [head][token] (16-bit).  bf16 pools run bf16
-    // MMAs on the stored rows; FP8 pools widen codes exactly to f16 and run
-    // f16 MMAs (q enters as f16 scaled by 2^-8, undone in the score scale).
+    // MMAs on the stored rows, with p as two bf16 terms (hi + lo, two PV MMAs
+    // on the same V fragments) so that it keeps about 16 significant bits;
+    // FP8 pools widen codes exactly to f16 and run f16 MMAs with p in f16 (q
+    // enters as f16 scaled by 2^-8, undone in the score scale).
     constexpr bool kF8 = sizeof(E) == 1;
     constexpr int NT = T / 16;  // 16-token tiles per stage (bf16 1, FP8 2)
     constexpr int kPS = LT::kPStride;
@@ -705,7 +710,9 @@ __global__ void __launch_bounds__(32 * 12, 1) decode_split_kernel(const DecodeAr
     const int qr = lane >> 2, kq = lane & 3;
     const bool v0 = 2 * kq < G, v1 = 2 * kq + 1 < G;
     const float sl = kF8 ? a.scale_log2 * 256.f : a.scale_log2;
-    uint16_t* pw = reinterpret_cast<uint16_t*>(smem + L.psm_off) + g * (8 * kPS);
+    constexpr bool kSplitP = LT::kSplitP;
+    uint16_t* pw = reinterpret_cast<uint16_t*>(smem + L.psm_off) + g * (8 * kPS) * (kSplitP ? 2 : 1);
+    uint16_t* pw_lo = pw + 8 * kPS;  // low bf16 terms (bf16 pools)
     const uint32_t ring_s = smem_u32(ring);
     // ldmatrix row of this lane: K (plain) matrices are (tokens 0-7 | 8-15) x
     // (first | second 16 bytes); V (transposed) matrices are (first | second
@@ -899,9 +906,15 @@ __global__ void __launch_bounds__(32 * 12, 1) decode_split_kernel(const DecodeAr
             acc[mt][3] *= al1;
           }
         }
-        auto to16 = [](float x) -> uint16_t {
-          if constexpr (kF8) return __half_as_ushort(__float2half_rn(x));
-          else return __bfloat16_as_ushort(__float2bfloat16_rn(x));
+        // p into the buffers: f16 (FP8 pools), or bf16 hi and lo terms.
+        auto put = [&](int i, float x) {
+          if constexpr (kF8) {
+            pw[i] = __half_as_ushort(__float2half_rn(x));
+          } else {
+            const __nv_bfloat16 h = __float2bfloat16_rn(x);
+            pw[i] = __bfloat16_as_ushort(h);
+            if constexpr (kSplitP) pw_lo[i] = __bfloat16_as_ushort(__float2bfloat16_rn(x - __bfloat162float(h)));
+          }
         };
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
@@ -910,24 +923,28 @@ __global__ void __launch_bounds__(32 * 12, 1) decode_split_kernel(const DecodeAr
           l0 += p00 + p10;
           l1 += p01 + p11;
           if (v0) {
-            pw[(2 * kq) * kPS + 16 * nt + qr] = to16(p00);
-            pw[(2 * kq) * kPS + 16 * nt + qr + 8] = to16(p10);
+            put((2 * kq) * kPS + 16 * nt + qr, p00);
+            put((2 * kq) * kPS + 16 * nt + qr + 8, p10);
           }
           if (v1) {
-            pw[(2 * kq + 1) * kPS + 16 * nt + qr] = to16(p01);
-            pw[(2 * kq + 1) * kPS + 16 * nt + qr + 8] = to16(p11);
+            put((2 * kq + 1) * kPS + 16 * nt + qr, p01);
+            put((2 * kq + 1) * kPS + 16 * nt + qr + 8, p11);
           }
         }
         __syncwarp();
         // P^T B fragments: b0 = p of head qr at tokens 2kq, 2kq + 1 of the
-        // tile; b1 at + 8.
-        uint32_t pb[NT][2];
+        // tile; b1 at + 8 (pl: the low terms).
+        uint32_t pb[NT][2], pl[NT][2];
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
-          pb[nt][0] = pb[nt][1] = 0u;
+          pb[nt][0] = pb[nt][1] = pl[nt][0] = pl[nt][1] = 0u;
           if (qr < G) {
             pb[nt][0] = *reinterpret_cast<const uint32_t*>(pw + qr * kPS + 16 * nt + 2 * kq);
             pb[nt][1] = *reinterpret_cast<const uint32_t*>(pw + qr * kPS + 16 * nt + 2 * kq + 8);
+            if constexpr (kSplitP) {
+              pl[nt][0] = *reinterpret_cast<const uint32_t*>(pw_lo + qr * kPS + 16 * nt + 2 * kq);
+              pl[nt][1] = *reinterpret_cast<const uint32_t*>(pw_lo + qr * kPS + 16 * nt + 2 * kq + 8);
+            }
           }
         }
         __syncwarp();
@@ -977,6 +994,7 @@ __global__ void __launch_bounds__(32 * 12, 1) decode_split_kernel(const DecodeAr
                 f[3] &= mhi;
               }
               mma16816<false>(acc[mt], f, pb[nt][0], pb[nt][1]);
+              if constexpr (kSplitP) mma16816<false>(acc[mt], f, pl[nt][0], pl[nt][1]);
             }
           }
         };

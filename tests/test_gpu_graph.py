@@ -9,9 +9,13 @@ one captured graph serves any batch up to its size.  Here each graph is
 replayed twice with different real batches and the real rows are compared
 with the float64 oracle.
 """
+import dataclasses
+
 import numpy as np
 import pytest
 import torch
+
+import oracle
 
 from gpu_helpers import device_pool, from_dev, i32, oracle_decode, to_dev, tol_check
 from paged_kv_gqa_scatter_b200 import api
@@ -115,7 +119,6 @@ def test_fused_store_then_cascade_decode_in_graph():
     replayed with two different qkv inputs in the same fixed buffer: each
     replay equals (bit for bit) the same two calls run eagerly, and the
     eager result matches the oracle's store and decode."""
-    import oracle
     gd = W.grouped_decode(groups=((128, 6), (700, 10)), max_suffix=200, seed=61)
     d = gd.decode
     Hq, Hkv, B = d.num_q_heads, d.pool.num_kv_heads, d.batch
@@ -192,3 +195,46 @@ def test_fp8_store_and_decode_in_graph():
         torch.cuda.synchronize()
         assert torch.equal(de.out, dg.out)
     assert int(de.err.item()) == 0 and int(dg.err.item()) == 0
+
+
+@pytest.mark.parametrize("fp8", [False, True])
+def test_paged_decode_in_graph_with_new_queries(fp8):
+    """Page size 16 (page-box stages, tensor maps passed as kernel parameters)
+    captured once and replayed with two different query sets: each replay
+    must match the oracle on the queries in the buffer at replay time."""
+    base = W.decode_paged_small(page_size=16, seq_lens=(1, 15, 17, 33, 300, 1029, 47), seed=1700)
+    wl = W.with_fp8_pool(base, seed=71) if fp8 else base
+    pool = device_pool(wl.pool, wl.k_planes, wl.v_planes, layers=[0])
+    table = api.PageTable(i32(wl.page_table))
+    q = to_dev(wl.q, W.BF16)
+    k_new, v_new = to_dev(wl.k_new, W.BF16), to_dev(wl.v_new, W.BF16)
+    loc, sl, ti = i32(wl.out_loc), i32(wl.seq_lens), i32(wl.table_idx)
+    out = torch.zeros_like(q)
+    ws = api.decode_workspace(wl.batch, wl.num_q_heads)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+
+    def step():
+        api.store_kv(pool, 0, k_new, v_new, loc, err)
+        api.decode_attn(pool, 0, q, table, ti, sl, out, ws, scale=wl.scale, dev_err=err)
+
+    g = _capture(step)
+    rng = np.random.default_rng(17)
+    for trial in range(2):
+        qs = wl.q if trial == 0 else W.draw_values(rng, wl.q.shape, W.BF16)
+        q.copy_(to_dev(qs, W.BF16))
+        out.fill_(0)
+        g.replay()
+        torch.cuda.synchronize()
+        wq = dataclasses.replace(wl, q=qs)
+        if fp8:
+            kp = {l: a.copy() for l, a in wl.k_planes.items()}
+            vp = {l: a.copy() for l, a in wl.v_planes.items()}
+            oracle.store_kv_fp8(kp, vp, 0, wl.k_new, wl.v_new, wl.out_loc, wl.pool.num_kv_heads, 128,
+                                wl.pool.k_scale, wl.pool.v_scale)
+            exp = oracle.decode_attn(qs, oracle.dequant_planes(kp, wl.pool.k_scale, [0]),
+                                     oracle.dequant_planes(vp, wl.pool.v_scale, [0]), 0, wl.page_table,
+                                     wl.table_idx, wl.seq_lens, 16, wl.scale)
+        else:
+            exp, _ = oracle_decode(wq)
+        tol_check(from_dev(out), exp, W.BF16, f"paged decode in a graph, trial {trial}, fp8={fp8}")
+    assert int(err.item()) == 0
