@@ -252,21 +252,6 @@ __device__ __forceinline__ void transpose_reduce(float (&v)[V], int d) {
 
 constexpr int ilog2c(int x) { return x <= 1 ? 0 : 1 + ilog2c(x / 2); }
 
-// 16 consecutive E4M3 codes (one 16-byte shared-memory load) -> two groups of
-// 8 floats (exact: code -> half -> float).
-__device__ __forceinline__ void load16_e4m3(const uint8_t* p, float2 (&lo)[4], float2 (&hi)[4]) {
-  const uint4 w = *reinterpret_cast<const uint4*>(p);
-  const uint32_t u[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const __half2_raw a = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(u[i] & 0xffffu), __NV_E4M3);
-    const __half2_raw b = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(u[i] >> 16), __NV_E4M3);
-    float2 (&dst)[4] = i < 2 ? lo : hi;
-    dst[(2 * i) & 3] = __half22float2(*reinterpret_cast<const __half2*>(&a));
-    dst[(2 * i + 1) & 3] = __half22float2(*reinterpret_cast<const __half2*>(&b));
-  }
-}
-
 // p values of query heads 0..G-1 for one token, from the warp's p buffer.
 template <int G>
 __device__ __forceinline__ void load_p(const float* src, float (&p)[G]) {
@@ -296,17 +281,16 @@ __global__ void __launch_bounds__(32 * 12, 1) decode_split_kernel(const DecodeAr
                                                                  const __grid_constant__ CUtensorMap kmap,
                                                                  const __grid_constant__ CUtensorMap vmap) {
   constexpr int T = DecodeTraits<E>::kTokensPerStage;
+  // Shape of the CUDA-core consumers (fp32 pools; the tensor-core consumers
+  // set their own below).
   constexpr int SUB = (64 / G < T) ? 64 / G : T;  // tokens per softmax sub-step
   constexpr int HALF = SUB / 2;                    // PV: tokens per lane per sub-step
   // Scores: D lanes share a token (each owns 16/D units of 8 dims), TL =
   // 32/D tokens are in flight per warp step, and a lane keeps V = SPL*G
   // partial sums per sub-step.  D = 8 halves the reduction of D = 16; wide
   // groups (G = 8, whose q would not fit in registers) keep D = 16.  A lane's
-  // units are dims 8d and 64 + 8d (16-byte loads of bf16 or fp32 rows), or,
-  // for FP8 rows, the 16 consecutive dims 16d .. 16d + 15, read as one
-  // 16-byte load (so that the 8 lanes of a token read 128 contiguous bytes).
+  // units are dims 8d and 64 + 8d (16-byte loads of bf16 or fp32 rows).
   constexpr int D = G >= 8 ? 16 : 8;
-  constexpr bool kWideFp8 = sizeof(E) == 1 && D == 8;
   constexpr int TL = 32 / D;
   constexpr int UPL = 16 / D;                      // 8-element units per lane
   constexpr int SPL = SUB / TL;                    // tokens per lane per sub-step
@@ -1066,7 +1050,7 @@ __global__ void __launch_bounds__(32 * 12, 1) decode_split_kernel(const DecodeAr
       }
     }
   } else {
-  // ============================= consumers ==================================
+  // ===================== consumers (CUDA cores, fp32 pools) ===================
   // Scores use the token-group lane map (tl, d) = (lane / D, lane % D); the
   // PV product uses (half, c) = (lane / 16, lane % 16): lane c owns dims
   // 8c .. 8c+7 and half picks even or odd tokens.  The p values pass from the
@@ -1085,7 +1069,7 @@ __global__ void __launch_bounds__(32 * 12, 1) decode_split_kernel(const DecodeAr
   auto head_lane = [](int hh) { return hh * LPH; };
   float* pw = psm + g * SUB * G;  // this warp's p buffer [SUB][G]
   // First dim of this lane's score unit m.
-  auto unit_dim = [&](int m) { return kWideFp8 ? 16 * d + 8 * m : 8 * (d + D * m); };
+  auto unit_dim = [&](int m) { return 8 * (d + D * m); };
   const IO* qbase = static_cast<const IO*>(a.q);
   IO* obase = static_cast<IO*>(a.out);
   int64_t s = 0;
@@ -1145,14 +1129,9 @@ __global__ void __launch_bounds__(32 * 12, 1) decode_split_kernel(const DecodeAr
           const int t = sub + TL * i + tl;
           float2 acc[G];
           float2 kw[UPL][4];
-          if constexpr (kWideFp8) {
-            load16_e4m3(kst + t * RS + g * kHeadDim + 16 * d, kw[0], kw[UPL - 1]);
-          } else {
 #pragma unroll
-            for (int m = 0; m < UPL; ++m)
-              load8<E>(reinterpret_cast<const E*>(kst + t * RS + (g * kHeadDim + unit_dim(m)) * ESZ),
-                       kw[m]);
-          }
+          for (int m = 0; m < UPL; ++m)
+            load8<E>(reinterpret_cast<const E*>(kst + t * RS + (g * kHeadDim + unit_dim(m)) * ESZ), kw[m]);
 #pragma unroll
           for (int m = 0; m < UPL; ++m) {
             const float2 (&k2)[4] = kw[m];
@@ -1248,15 +1227,6 @@ __global__ void __launch_bounds__(32 * 12, 1) decode_split_kernel(const DecodeAr
         o2[hh][e].x += __shfl_xor_sync(0xffffffffu, o2[hh][e].x, 16);
         o2[hh][e].y += __shfl_xor_sync(0xffffffffu, o2[hh][e].y, 16);
       }
-    }
-    if constexpr (sizeof(E) == 1) {  // FP8 pool: V codes stand for code * v_scale
-#pragma unroll
-      for (int hh = 0; hh < G; ++hh)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          o2[hh][e].x *= a.v_scale;
-          o2[hh][e].y *= a.v_scale;
-        }
     }
 #pragma unroll
     for (int hh = 0; hh < G; ++hh) {
