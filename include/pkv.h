@@ -293,7 +293,8 @@ int pkv_gather_kv(const pkv_pool* pool, int32_t layer, const pkv_page_table* tab
  *   num_q_heads) bytes, 16-byte aligned, owned by the caller, not shared by
  *   calls that may overlap on the GPU.
  * Supported: head_dim 128, num_kv_heads 1..8, num_q_heads/num_kv_heads in
- *   {1, 2, 4, 8}.  seq_lens[r] < 1 writes a zero row and sets
+ *   {1, 2, 4, 8}, and 16 on bf16 and FP8 pools (extend and cascade decode
+ *   stop at 8).  seq_lens[r] < 1 writes a zero row and sets
  *   PKV_DEV_ERR_EMPTY_CONTEXT.  batch == 0 is a no-op.
  * The work is split across the context (split-KV): one persistent grid
  * walks (request, chunk) items, then a second kernel merges the chunks of

@@ -76,10 +76,13 @@ int check_table(const pkv_page_table* t, TableView* out) {
   return PKV_OK;
 }
 
-int check_heads(const pkv_pool* p, int32_t num_q_heads) {
+// Head counts: Hkv <= 8 and G = Hq / Hkv in {1, 2, 4, 8}; plain decode on a
+// bf16 or E4M3 pool also takes G = 16 (two 8-head column tiles).
+int check_heads(const pkv_pool* p, int32_t num_q_heads, bool group16_ok = false) {
   if (p->num_kv_heads > 8) return PKV_ERR_UNSUPPORTED;
   if (num_q_heads < 1 || num_q_heads % p->num_kv_heads != 0) return PKV_ERR_INVALID_ARG;
   const int G = num_q_heads / p->num_kv_heads;
+  if (G == 16 && group16_ok && p->dtype != PKV_DTYPE_F32) return PKV_OK;
   if (G != 1 && G != 2 && G != 4 && G != 8) return PKV_ERR_UNSUPPORTED;
   return PKV_OK;
 }
@@ -194,7 +197,7 @@ int pkv_decode_attn(const pkv_pool* pool, int32_t layer, const void* q, int32_t 
   TableView tv;
   int st = check_pool(pool, layer, &pv);
   if (st != PKV_OK) return st;
-  st = check_heads(pool, num_q_heads);
+  st = check_heads(pool, num_q_heads, /*group16_ok=*/true);
   if (st != PKV_OK) return st;
   if (batch < 0) return PKV_ERR_INVALID_ARG;
   if (batch == 0) return PKV_OK;

@@ -137,7 +137,9 @@ template <typename E>
 struct DecodeLayoutTraits {
   static constexpr bool kMma = sizeof(E) != 4;
   static constexpr int kRowPad = kMma ? 16 : 0;
-  static constexpr int kPStride = 40;  // p buffer row (16-bit entries) per head, 32 tokens + pad
+  // p buffer row per head (16-bit entries): a stage's tokens + 8 (the pad
+  // spreads the rows' writes and reads over different banks).
+  static constexpr int kPStride = DecodeTraits<E>::kTokensPerStage + 8;
   // Producer warps.  One warp issuing one bulk copy per row tops out near 3 G
   // copies/s (measured on B200: 3.1 TB/s at 1 KB rows); four warps, each
   // copying one plane for every other token, reach the HBM bandwidth.
@@ -146,8 +148,8 @@ struct DecodeLayoutTraits {
   // about 2^-17 relative), in two buffers; f16 (FP8 pools) keeps 11 bits.
   static constexpr bool kSplitP = kMma && sizeof(E) == 2;
   template <int G>
-  static constexpr int psm_per_warp() {
-    return kMma ? 8 * kPStride * 2 * (kSplitP ? 2 : 1) : 4 * DecodeTraits<E>::kTokensPerStage * G;
+  static constexpr int psm_per_warp() {  // rows for 8 heads per column tile
+    return kMma ? 8 * ((G + 7) / 8) * kPStride * 2 * (kSplitP ? 2 : 1) : 4 * DecodeTraits<E>::kTokensPerStage * G;
   }
 };
 
@@ -672,11 +674,13 @@ __global__ void __launch_bounds__(32 * 12, 1) decode_split_kernel(const DecodeAr
 
   if constexpr (LT::kMma) {
     // ======================= consumers (tensor cores) =========================
-    // Per 16-token sub-step, with the GQA group as the N dimension:
+    // Per 16-token tile, with the GQA group as the N dimension (one column
+    // tile of 8 heads, two at G = 16):
     //   S^T (16 tokens x 8 heads)  = K (16 x 128) . Q^T (128 x 8)  8 MMAs
     //   O^T (128 dims x 8 heads)  += V^T (128 x 16) . P^T (16 x 8)  8 MMAs
     // Lane (qr, kq) = (lane / 4, lane % 4) holds scores of tokens qr, qr + 8
-    // and output columns for heads 2kq, 2kq + 1 (columns >= G are padding),
+    // and output columns for heads 2kq, 2kq + 1 of each column tile (columns
+    // >= G are padding),
     // so its softmax state (max, sum) covers exactly the heads whose output it
     // accumulates.  P passes from the score layout to the PV B fragment
     // through the warp's p buffer [head][token] (16-bit).  bf16 pools run bf16
@@ -692,11 +696,14 @@ __global__ void __launch_bounds__(32 * 12, 1) decode_split_kernel(const DecodeAr
     const int g = warp - kProd;  // KV head
     if (g >= ncons) return;
     const int qr = lane >> 2, kq = lane & 3;
-    const bool v0 = 2 * kq < G, v1 = 2 * kq + 1 < G;
+    // The group's heads form NH column tiles of 8 (NH = 2 at G = 16); in tile
+    // h this lane's columns are heads 8h + 2kq and 8h + 2kq + 1.
+    constexpr int NH = (G + 7) / 8;
+    auto hv = [&](int h, int hs) { return 8 * h + 2 * kq + hs < G; };
     const float sl = kF8 ? a.scale_log2 * 256.f : a.scale_log2;
     constexpr bool kSplitP = LT::kSplitP;
-    uint16_t* pw = reinterpret_cast<uint16_t*>(smem + L.psm_off) + g * (8 * kPS) * (kSplitP ? 2 : 1);
-    uint16_t* pw_lo = pw + 8 * kPS;  // low bf16 terms (bf16 pools)
+    uint16_t* pw = reinterpret_cast<uint16_t*>(smem + L.psm_off) + g * (8 * NH * kPS) * (kSplitP ? 2 : 1);
+    uint16_t* pw_lo = pw + 8 * NH * kPS;  // low bf16 terms (bf16 pools)
     const uint32_t ring_s = smem_u32(ring);
     // ldmatrix row of this lane: K (plain) matrices are (tokens 0-7 | 8-15) x
     // (first | second 16 bytes); V (transposed) matrices are (first | second
@@ -719,31 +726,42 @@ __global__ void __launch_bounds__(32 * 12, 1) decode_split_kernel(const DecodeAr
       // Q^T B fragments, 16 dims per MMA: b0 = dims k, k + 1 and b1 = dims
       // k + 8, k + 9 (k = 2 kq) of head qr.  FP8 rows use the dim order of
       // their K fragments instead: b0 = dims 4kq, 4kq + 1, b1 = 4kq + 2, 4kq + 3.
-      uint32_t qb[8][2];
-      if (qr < G) {
-        const IO* qrow = qbase + ((int64_t)r * a.hq + g * G + qr) * kHeadDim;
+      uint32_t qb[NH][8][2];
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          if constexpr (kF8) {
-            const uint2 w = *reinterpret_cast<const uint2*>(qrow + 16 * c + 4 * kq);
-            qb[c][0] = pack_f16x2(bf16_lo(w.x) * kQPre, bf16_hi(w.x) * kQPre);
-            qb[c][1] = pack_f16x2(bf16_lo(w.y) * kQPre, bf16_hi(w.y) * kQPre);
-          } else {
-            qb[c][0] = *reinterpret_cast<const uint32_t*>(qrow + 16 * c + 2 * kq);
-            qb[c][1] = *reinterpret_cast<const uint32_t*>(qrow + 16 * c + 2 * kq + 8);
+      for (int h = 0; h < NH; ++h) {
+        if (8 * h + qr < G) {
+          const IO* qrow = qbase + ((int64_t)r * a.hq + g * G + 8 * h + qr) * kHeadDim;
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            if constexpr (kF8) {
+              const uint2 w = *reinterpret_cast<const uint2*>(qrow + 16 * c + 4 * kq);
+              qb[h][c][0] = pack_f16x2(bf16_lo(w.x) * kQPre, bf16_hi(w.x) * kQPre);
+              qb[h][c][1] = pack_f16x2(bf16_lo(w.y) * kQPre, bf16_hi(w.y) * kQPre);
+            } else {
+              qb[h][c][0] = *reinterpret_cast<const uint32_t*>(qrow + 16 * c + 2 * kq);
+              qb[h][c][1] = *reinterpret_cast<const uint32_t*>(qrow + 16 * c + 2 * kq + 8);
+            }
           }
-        }
-      } else {
+        } else {
 #pragma unroll
-        for (int c = 0; c < 8; ++c) qb[c][0] = qb[c][1] = 0u;
+          for (int c = 0; c < 8; ++c) qb[h][c][0] = qb[h][c][1] = 0u;
+        }
       }
-      float acc[8][4];
+      float acc[8][NH][4];
 #pragma unroll
       for (int mt = 0; mt < 8; ++mt)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) acc[mt][e] = 0.f;
-      float l0 = 0.f, l1 = 0.f;              // this lane's share of the sums of p
-      float m0 = -INFINITY, m1 = -INFINITY;  // running max of heads 2kq, 2kq + 1 (log2 domain)
+        for (int h = 0; h < NH; ++h)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) acc[mt][h][e] = 0.f;
+      float lsum[NH][2], mrun[NH][2];  // per column head: this lane's share of the sum of p; running max (log2)
+#pragma unroll
+      for (int h = 0; h < NH; ++h)
+#pragma unroll
+        for (int hs = 0; hs < 2; ++hs) {
+          lsum[h][hs] = 0.f;
+          mrun[h][hs] = -INFINITY;
+        }
 
       // Stages: T tokens each (row copies), or NT groups of 16 table columns
       // aligned to 16 (page boxes; a piece's first and last groups may be
@@ -817,10 +835,14 @@ __global__ void __launch_bounds__(32 * 12, 1) decode_split_kernel(const DecodeAr
         };
         // ---- scores: NT independent 16-token tiles, each with two
         // accumulators (even and odd 16-dim chunks) to halve the MMA chain.
-        float sc[NT][4];
+        float sc[NT][NH][4];
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
-          float se[4] = {0.f, 0.f, 0.f, 0.f}, so[4] = {0.f, 0.f, 0.f, 0.f};
+          float se[NH][4], so[NH][4];
+#pragma unroll
+          for (int h = 0; h < NH; ++h)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) se[h][e] = so[h][e] = 0.f;
           if (hi_t[nt] > lo_t[nt]) {
             if constexpr (kF8) {
 #pragma unroll
@@ -830,8 +852,11 @@ __global__ void __launch_bounds__(32 * 12, 1) decode_split_kernel(const DecodeAr
                 // w[0], w[1]: tokens 0-7, 8-15 of 16-dim chunk 2cp; w[2], w[3]: chunk 2cp + 1.
                 const uint32_t f0[4] = {lo_f16x2(w[0]), lo_f16x2(w[1]), hi_f16x2(w[0]), hi_f16x2(w[1])};
                 const uint32_t f1[4] = {lo_f16x2(w[2]), lo_f16x2(w[3]), hi_f16x2(w[2]), hi_f16x2(w[3])};
-                mma16816<true>(se, f0, qb[2 * cp][0], qb[2 * cp][1]);
-                mma16816<true>(so, f1, qb[2 * cp + 1][0], qb[2 * cp + 1][1]);
+#pragma unroll
+                for (int h = 0; h < NH; ++h) {
+                  mma16816<true>(se[h], f0, qb[h][2 * cp][0], qb[h][2 * cp][1]);
+                  mma16816<true>(so[h], f1, qb[h][2 * cp + 1][0], qb[h][2 * cp + 1][1]);
+                }
               }
             } else {
 #pragma unroll
@@ -839,98 +864,117 @@ __global__ void __launch_bounds__(32 * 12, 1) decode_split_kernel(const DecodeAr
                 uint32_t f0[4], f1[4];
                 ldsm_x4(k_addr(nt, c), f0);
                 ldsm_x4(k_addr(nt, c + 1), f1);
-                mma16816<false>(se, f0, qb[c][0], qb[c][1]);
-                mma16816<false>(so, f1, qb[c + 1][0], qb[c + 1][1]);
+#pragma unroll
+                for (int h = 0; h < NH; ++h) {
+                  mma16816<false>(se[h], f0, qb[h][c][0], qb[h][c][1]);
+                  mma16816<false>(so[h], f1, qb[h][c + 1][0], qb[h][c + 1][1]);
+                }
               }
             }
           }
 #pragma unroll
-          for (int e = 0; e < 4; ++e) sc[nt][e] = se[e] + so[e];
+          for (int h = 0; h < NH; ++h)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) sc[nt][h][e] = se[h][e] + so[h][e];
         }
-        // sc[nt] = S[token qr][head 2kq], S[qr][2kq + 1], S[qr + 8][2kq],
-        // S[qr + 8][2kq + 1] of tile nt; scaled to the log2 domain, masked.
-        float sv[NT][4];
-        float mx0 = -INFINITY, mx1 = -INFINITY;
+        // sc[nt][h] = S[token qr][head 8h + 2kq], S[qr][8h + 2kq + 1],
+        // S[qr + 8][8h + 2kq], S[qr + 8][8h + 2kq + 1] of tile nt; scaled to
+        // the log2 domain, masked.
+        float sv[NT][NH][4];
+        float mx[NH][2];
+#pragma unroll
+        for (int h = 0; h < NH; ++h) mx[h][0] = mx[h][1] = -INFINITY;
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
           const bool t0 = qr >= lo_t[nt] && qr < hi_t[nt];
           const bool t1 = qr + 8 >= lo_t[nt] && qr + 8 < hi_t[nt];
-          sv[nt][0] = (v0 && t0) ? sc[nt][0] * sl : -INFINITY;
-          sv[nt][1] = (v1 && t0) ? sc[nt][1] * sl : -INFINITY;
-          sv[nt][2] = (v0 && t1) ? sc[nt][2] * sl : -INFINITY;
-          sv[nt][3] = (v1 && t1) ? sc[nt][3] * sl : -INFINITY;
-          mx0 = fmaxf(mx0, fmaxf(sv[nt][0], sv[nt][2]));
-          mx1 = fmaxf(mx1, fmaxf(sv[nt][1], sv[nt][3]));
-        }
 #pragma unroll
-        for (int off = 4; off < 32; off <<= 1) {
-          mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
-          mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
-        }
-        // Lazy rescale: the max moves only when it grows by more than the
-        // threshold (p stays below 2^threshold, well inside f16 and bf16).
-        const bool need0 = mx0 > m0 + kRescaleThreshold, need1 = mx1 > m1 + kRescaleThreshold;
-        float al0 = 1.f, al1 = 1.f;
-        if (need0) {
-          al0 = exp2f(m0 - mx0);
-          m0 = mx0;
-          l0 *= al0;
-        }
-        if (need1) {
-          al1 = exp2f(m1 - mx1);
-          m1 = mx1;
-          l1 *= al1;
-        }
-        if (__any_sync(0xffffffffu, need0 || need1)) {
-#pragma unroll
-          for (int mt = 0; mt < 8; ++mt) {
-            acc[mt][0] *= al0;
-            acc[mt][2] *= al0;
-            acc[mt][1] *= al1;
-            acc[mt][3] *= al1;
+          for (int h = 0; h < NH; ++h) {
+            sv[nt][h][0] = (hv(h, 0) && t0) ? sc[nt][h][0] * sl : -INFINITY;
+            sv[nt][h][1] = (hv(h, 1) && t0) ? sc[nt][h][1] * sl : -INFINITY;
+            sv[nt][h][2] = (hv(h, 0) && t1) ? sc[nt][h][2] * sl : -INFINITY;
+            sv[nt][h][3] = (hv(h, 1) && t1) ? sc[nt][h][3] * sl : -INFINITY;
+            mx[h][0] = fmaxf(mx[h][0], fmaxf(sv[nt][h][0], sv[nt][h][2]));
+            mx[h][1] = fmaxf(mx[h][1], fmaxf(sv[nt][h][1], sv[nt][h][3]));
           }
         }
-        // p into the buffers: f16 (FP8 pools), or bf16 hi and lo terms.
+#pragma unroll
+        for (int off = 4; off < 32; off <<= 1)
+#pragma unroll
+          for (int h = 0; h < NH; ++h)
+#pragma unroll
+            for (int hs = 0; hs < 2; ++hs) mx[h][hs] = fmaxf(mx[h][hs], __shfl_xor_sync(0xffffffffu, mx[h][hs], off));
+        // Lazy rescale: the max moves only when it grows by more than the
+        // threshold (p stays below 2^threshold, well inside f16 and bf16).
+        float al[NH][2];
+        bool need_any = false;
+#pragma unroll
+        for (int h = 0; h < NH; ++h)
+#pragma unroll
+          for (int hs = 0; hs < 2; ++hs) {
+            al[h][hs] = 1.f;
+            if (mx[h][hs] > mrun[h][hs] + kRescaleThreshold) {
+              al[h][hs] = exp2f(mrun[h][hs] - mx[h][hs]);
+              mrun[h][hs] = mx[h][hs];
+              lsum[h][hs] *= al[h][hs];
+              need_any = true;
+            }
+          }
+        if (__any_sync(0xffffffffu, need_any)) {
+#pragma unroll
+          for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+            for (int h = 0; h < NH; ++h) {
+              acc[mt][h][0] *= al[h][0];
+              acc[mt][h][2] *= al[h][0];
+              acc[mt][h][1] *= al[h][1];
+              acc[mt][h][3] *= al[h][1];
+            }
+        }
+        // p into the buffers [head][token]: f16 (FP8 pools), or bf16 hi and
+        // lo terms.
         auto put = [&](int i, float x) {
           if constexpr (kF8) {
             pw[i] = __half_as_ushort(__float2half_rn(x));
           } else {
-            const __nv_bfloat16 h = __float2bfloat16_rn(x);
-            pw[i] = __bfloat16_as_ushort(h);
-            if constexpr (kSplitP) pw_lo[i] = __bfloat16_as_ushort(__float2bfloat16_rn(x - __bfloat162float(h)));
+            const __nv_bfloat16 hb = __float2bfloat16_rn(x);
+            pw[i] = __bfloat16_as_ushort(hb);
+            if constexpr (kSplitP) pw_lo[i] = __bfloat16_as_ushort(__float2bfloat16_rn(x - __bfloat162float(hb)));
           }
         };
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-          const float p00 = v0 ? exp2f(sv[nt][0] - m0) : 0.f, p10 = v0 ? exp2f(sv[nt][2] - m0) : 0.f;
-          const float p01 = v1 ? exp2f(sv[nt][1] - m1) : 0.f, p11 = v1 ? exp2f(sv[nt][3] - m1) : 0.f;
-          l0 += p00 + p10;
-          l1 += p01 + p11;
-          if (v0) {
-            put((2 * kq) * kPS + 16 * nt + qr, p00);
-            put((2 * kq) * kPS + 16 * nt + qr + 8, p10);
-          }
-          if (v1) {
-            put((2 * kq + 1) * kPS + 16 * nt + qr, p01);
-            put((2 * kq + 1) * kPS + 16 * nt + qr + 8, p11);
-          }
-        }
-        __syncwarp();
-        // P^T B fragments: b0 = p of head qr at tokens 2kq, 2kq + 1 of the
-        // tile; b1 at + 8 (pl: the low terms).
-        uint32_t pb[NT][2], pl[NT][2];
+        for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-          pb[nt][0] = pb[nt][1] = pl[nt][0] = pl[nt][1] = 0u;
-          if (qr < G) {
-            pb[nt][0] = *reinterpret_cast<const uint32_t*>(pw + qr * kPS + 16 * nt + 2 * kq);
-            pb[nt][1] = *reinterpret_cast<const uint32_t*>(pw + qr * kPS + 16 * nt + 2 * kq + 8);
-            if constexpr (kSplitP) {
-              pl[nt][0] = *reinterpret_cast<const uint32_t*>(pw_lo + qr * kPS + 16 * nt + 2 * kq);
-              pl[nt][1] = *reinterpret_cast<const uint32_t*>(pw_lo + qr * kPS + 16 * nt + 2 * kq + 8);
+          for (int h = 0; h < NH; ++h)
+#pragma unroll
+            for (int hs = 0; hs < 2; ++hs) {
+              if (!hv(h, hs)) continue;
+              const float p0 = exp2f(sv[nt][h][hs] - mrun[h][hs]);
+              const float p1 = exp2f(sv[nt][h][hs + 2] - mrun[h][hs]);
+              lsum[h][hs] += p0 + p1;
+              const int row = (8 * h + 2 * kq + hs) * kPS + 16 * nt;
+              put(row + qr, p0);
+              put(row + qr + 8, p1);
+            }
+        __syncwarp();
+        // P^T B fragments of column tile h: b0 = p of head 8h + qr at tokens
+        // 2kq, 2kq + 1 of the tile; b1 at + 8 (pl: the low terms).
+        uint32_t pb[NT][NH][2], pl[NT][NH][2];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+          for (int h = 0; h < NH; ++h) {
+            pb[nt][h][0] = pb[nt][h][1] = pl[nt][h][0] = pl[nt][h][1] = 0u;
+            if (8 * h + qr < G) {
+              const int row = (8 * h + qr) * kPS + 16 * nt + 2 * kq;
+              pb[nt][h][0] = *reinterpret_cast<const uint32_t*>(pw + row);
+              pb[nt][h][1] = *reinterpret_cast<const uint32_t*>(pw + row + 8);
+              if constexpr (kSplitP) {
+                pl[nt][h][0] = *reinterpret_cast<const uint32_t*>(pw_lo + row);
+                pl[nt][h][1] = *reinterpret_cast<const uint32_t*>(pw_lo + row + 8);
+              }
             }
           }
-        }
         __syncwarp();
         // ---- PV -------------------------------------------------------------
         // In a partial tile, tokens outside [lo, hi) are not this piece's
@@ -963,8 +1007,11 @@ __global__ void __launch_bounds__(32 * 12, 1) decode_split_kernel(const DecodeAr
                   fo[j] &= j < 2 ? mlo : mhi;
                 }
               }
-              mma16816<true>(acc[2 * pp], fe, pb[nt][0], pb[nt][1]);
-              mma16816<true>(acc[2 * pp + 1], fo, pb[nt][0], pb[nt][1]);
+#pragma unroll
+              for (int h = 0; h < NH; ++h) {
+                mma16816<true>(acc[2 * pp][h], fe, pb[nt][h][0], pb[nt][h][1]);
+                mma16816<true>(acc[2 * pp + 1][h], fo, pb[nt][h][0], pb[nt][h][1]);
+              }
             }
           } else {
 #pragma unroll
@@ -977,8 +1024,11 @@ __global__ void __launch_bounds__(32 * 12, 1) decode_split_kernel(const DecodeAr
                 f[2] &= mhi;
                 f[3] &= mhi;
               }
-              mma16816<false>(acc[mt], f, pb[nt][0], pb[nt][1]);
-              if constexpr (kSplitP) mma16816<false>(acc[mt], f, pl[nt][0], pl[nt][1]);
+#pragma unroll
+              for (int h = 0; h < NH; ++h) {
+                mma16816<false>(acc[mt][h], f, pb[nt][h][0], pb[nt][h][1]);
+                if constexpr (kSplitP) mma16816<false>(acc[mt][h], f, pl[nt][h][0], pl[nt][h][1]);
+              }
             }
           }
         };
@@ -997,57 +1047,61 @@ __global__ void __launch_bounds__(32 * 12, 1) decode_split_kernel(const DecodeAr
 
       // ---- finish the piece -------------------------------------------------
 #pragma unroll
-      for (int off = 4; off < 32; off <<= 1) {
-        l0 += __shfl_xor_sync(0xffffffffu, l0, off);
-        l1 += __shfl_xor_sync(0xffffffffu, l1, off);
-      }
+      for (int off = 4; off < 32; off <<= 1)
+#pragma unroll
+        for (int h = 0; h < NH; ++h)
+#pragma unroll
+          for (int hs = 0; hs < 2; ++hs) lsum[h][hs] += __shfl_xor_sync(0xffffffffu, lsum[h][hs], off);
       // Output dims of accumulator (mt, e): bf16 rows: 16 mt + qr (+ 8 for
       // e >= 2); FP8 rows: 32 (mt / 2) + 2 qr + (mt & 1) (+ 16 for e >= 2).
 #pragma unroll
-      for (int hs = 0; hs < 2; ++hs) {
-        if (!(hs == 0 ? v0 : v1)) continue;
-        const int h = g * G + 2 * kq + hs;
-        const float lsum = hs == 0 ? l0 : l1, mh = hs == 0 ? m0 : m1;
-        const float vs = kF8 ? a.v_scale : 1.f;
-        if (whole) {
-          const float inv = lsum > 0.f ? vs / lsum : 0.f;
-          IO* orow = obase + ((int64_t)r * a.hq + h) * kHeadDim;
-          if constexpr (kF8) {
+      for (int h = 0; h < NH; ++h)
 #pragma unroll
-            for (int pp = 0; pp < 4; ++pp) {
+        for (int hs = 0; hs < 2; ++hs) {
+          if (!hv(h, hs)) continue;
+          const int head = g * G + 8 * h + 2 * kq + hs;
+          const float ls = lsum[h][hs], mh = mrun[h][hs];
+          const float vs = kF8 ? a.v_scale : 1.f;
+          if (whole) {
+            const float inv = ls > 0.f ? vs / ls : 0.f;
+            IO* orow = obase + ((int64_t)r * a.hq + head) * kHeadDim;
+            if constexpr (kF8) {
 #pragma unroll
-              for (int up = 0; up < 2; ++up) {
-                const uint32_t w = pack_bf16x2(acc[2 * pp][hs + 2 * up] * inv, acc[2 * pp + 1][hs + 2 * up] * inv);
-                *reinterpret_cast<uint32_t*>(orow + 32 * pp + 16 * up + 2 * qr) = w;
+              for (int pp = 0; pp < 4; ++pp) {
+#pragma unroll
+                for (int up = 0; up < 2; ++up) {
+                  const uint32_t w =
+                      pack_bf16x2(acc[2 * pp][h][hs + 2 * up] * inv, acc[2 * pp + 1][h][hs + 2 * up] * inv);
+                  *reinterpret_cast<uint32_t*>(orow + 32 * pp + 16 * up + 2 * qr) = w;
+                }
+              }
+            } else {
+#pragma unroll
+              for (int mt = 0; mt < 8; ++mt) {
+                orow[16 * mt + qr] = __float2bfloat16_rn(acc[mt][h][hs] * inv);
+                orow[16 * mt + qr + 8] = __float2bfloat16_rn(acc[mt][h][hs + 2] * inv);
               }
             }
           } else {
+            const int64_t id = static_cast<int64_t>(blockIdx.x) + r;
+            float* op = a.ws_o + (id * a.hq + head) * kHeadDim;
+            if constexpr (kF8) {
 #pragma unroll
-            for (int mt = 0; mt < 8; ++mt) {
-              orow[16 * mt + qr] = __float2bfloat16_rn(acc[mt][hs] * inv);
-              orow[16 * mt + qr + 8] = __float2bfloat16_rn(acc[mt][hs + 2] * inv);
+              for (int pp = 0; pp < 4; ++pp)
+#pragma unroll
+                for (int up = 0; up < 2; ++up)
+                  *reinterpret_cast<float2*>(op + 32 * pp + 16 * up + 2 * qr) =
+                      make_float2(acc[2 * pp][h][hs + 2 * up] * vs, acc[2 * pp + 1][h][hs + 2 * up] * vs);
+            } else {
+#pragma unroll
+              for (int mt = 0; mt < 8; ++mt) {
+                op[16 * mt + qr] = acc[mt][h][hs];
+                op[16 * mt + qr + 8] = acc[mt][h][hs + 2];
+              }
             }
+            if (qr == 0) a.ws_ml[id * a.hq + head] = make_float2(mh, ls);
           }
-        } else {
-          const int64_t id = static_cast<int64_t>(blockIdx.x) + r;
-          float* op = a.ws_o + (id * a.hq + h) * kHeadDim;
-          if constexpr (kF8) {
-#pragma unroll
-            for (int pp = 0; pp < 4; ++pp)
-#pragma unroll
-              for (int up = 0; up < 2; ++up)
-                *reinterpret_cast<float2*>(op + 32 * pp + 16 * up + 2 * qr) =
-                    make_float2(acc[2 * pp][hs + 2 * up] * vs, acc[2 * pp + 1][hs + 2 * up] * vs);
-          } else {
-#pragma unroll
-            for (int mt = 0; mt < 8; ++mt) {
-              op[16 * mt + qr] = acc[mt][hs];
-              op[16 * mt + qr + 8] = acc[mt][hs + 2];
-            }
-          }
-          if (qr == 0) a.ws_ml[id * a.hq + h] = make_float2(mh, lsum);
         }
-      }
     }
   } else {
   // ===================== consumers (CUDA cores, fp32 pools) ===================
@@ -1492,6 +1546,7 @@ cudaError_t launch_decode(const PoolView& pool, const TableView& t, const void* 
       case 2: return launch_decode_t<__nv_fp8_e4m3, 2>(a, grid, s, cascade);
       case 4: return launch_decode_t<__nv_fp8_e4m3, 4>(a, grid, s, cascade);
       case 8: return launch_decode_t<__nv_fp8_e4m3, 8>(a, grid, s, cascade);
+      case 16: return launch_decode_t<__nv_fp8_e4m3, 16>(a, grid, s, cascade);
     }
   } else if (pool.dtype == PKV_DTYPE_BF16) {
     switch (G) {
@@ -1499,6 +1554,7 @@ cudaError_t launch_decode(const PoolView& pool, const TableView& t, const void* 
       case 2: return launch_decode_t<__nv_bfloat16, 2>(a, grid, s, cascade);
       case 4: return launch_decode_t<__nv_bfloat16, 4>(a, grid, s, cascade);
       case 8: return launch_decode_t<__nv_bfloat16, 8>(a, grid, s, cascade);
+      case 16: return launch_decode_t<__nv_bfloat16, 16>(a, grid, s, cascade);
     }
   } else {
     switch (G) {

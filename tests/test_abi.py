@@ -94,6 +94,18 @@ def test_host_validation_rejects_bad_arguments():
     # empty batch is a no-op
     assert lib.pkv_decode_attn(P(_pool()), 0, dummy, 16, P(t), dummy, dummy, 0, 0.1, dummy, dummy,
                                0, None, None) == 0
+    # GQA group 16: decode on bf16 and E4M3 pools passes the head check (an empty
+    # batch then launches nothing); fp32 pools, extend and groups of 32 are not built
+    assert lib.pkv_decode_attn(P(_pool()), 0, dummy, 128, P(t), dummy, dummy, 0, 0.1, dummy, dummy,
+                               0, None, None) == 0
+    assert lib.pkv_decode_attn(P(_pool(dtype=2, k_scale=0.5, v_scale=0.5)), 0, dummy, 128, P(t), dummy, dummy, 0, 0.1,
+                               dummy, dummy, 0, None, None) == 0
+    assert lib.pkv_decode_attn(P(_pool(dtype=1, layer_stride=64 * 1024)), 0, dummy, 128, P(t), dummy, dummy, 2,
+                               0.1, dummy, dummy, 1 << 20, None, None) == 2
+    assert lib.pkv_decode_attn(P(_pool()), 0, dummy, 256, P(t), dummy, dummy, 2, 0.1, dummy, dummy,
+                               1 << 20, None, None) == 2
+    assert lib.pkv_extend_attn(P(_pool()), 0, dummy, 128, P(t), dummy, dummy, dummy, dummy, 2, 10,
+                               5, 0.1, dummy, None, 0, None, None) == 2
     # bad table (row stride < cols)
     tb = _lib.PkvPageTable(entries=dummy, rows=4, cols=64, row_stride=8)
     assert lib.pkv_extend_attn(P(_pool()), 0, dummy, 16, P(tb), dummy, dummy, dummy, dummy, 2, 10,

@@ -194,6 +194,21 @@ def test_fp8_decode_nan_codes_in_unreferenced_slots():
     scale_check(from_dev(d.out), exp, "fp8 decode, NaN codes in unreferenced slots")
 
 
+@pytest.mark.parametrize("page_size", [1, 16])
+def test_fp8_decode_group_16(page_size):
+    """E4M3 pool, 128 query heads over 8 KV heads (G = 16)."""
+    wl = W.with_fp8_pool(W.decode_paged_small(page_size=page_size, num_q_heads=128, num_kv_heads=8,
+                                              seed=1900 + page_size), seed=19)
+    d = DeviceDecode(wl)
+    d.run()
+    torch.cuda.synchronize()
+    assert int(d.err.item()) == 0
+    kp, vp = _oracle_store(wl)
+    exp = _oracle_decode(wl, kp, vp)
+    tol_check(from_dev(d.out), exp, W.BF16, f"fp8 decode G=16 P={page_size}")
+    scale_check(from_dev(d.out), exp, f"fp8 decode G=16 P={page_size}")
+
+
 def test_fp8_rope_store():
     wl = W.rope_store_step(W.BF16, seed=31)
     hq, hkv = wl.num_q_heads, wl.pool.num_kv_heads

@@ -185,6 +185,20 @@ def test_decode_nan_in_unreferenced_slots(dtype, page_size, hq, hkv):
     assert _err(d.err) == 0
 
 
+@pytest.mark.parametrize("page_size,hq,hkv", [(1, 16, 1), (1, 64, 4), (16, 128, 8), (16, 32, 2)])
+def test_decode_group_16(page_size, hq, hkv):
+    """GQA groups of 16 query heads per KV head (two 8-head column tiles of
+    the tensor-core consumers), row copies and page boxes, ragged lengths
+    spread over many CTAs so that most requests go through the merge."""
+    wl = W.decode_paged_small(dtype=W.BF16, page_size=page_size, num_q_heads=hq, num_kv_heads=hkv,
+                              seed=1800 + hq + page_size)
+    d = DeviceDecode(wl)
+    d.run()
+    exp, _ = oracle_decode(wl)
+    tol_check(from_dev(d.out), exp, W.BF16, f"decode G=16 P={page_size} hq={hq} hkv={hkv}")
+    assert _err(d.err) == 0
+
+
 def test_decode_one_token_returns_v_exactly():
     wl = W.decode_small(seq_lens=(1, 1, 1))
     d = DeviceDecode(wl)
