@@ -25,6 +25,7 @@
 #include <cuda_bf16.h>
 
 #include <algorithm>
+#include <cmath>
 
 #include "common.cuh"
 #include "launch.h"
@@ -102,6 +103,49 @@ cudaError_t launch_cascade_prep(const int32_t* group_offsets, const int32_t* gro
   return cudaGetLastError();
 }
 
+// The prefix pass (tensor cores) and the suffix pass (HBM) use different
+// units, so when the prefix pass is small enough they run side by side: the
+// prefix pass on an auxiliary stream with about 43% of the SMs' worth of
+// CTAs, the suffix pass on the caller's stream with the remaining SMs as its
+// persistent grid, joined by an event before the merge.  (Inside a CUDA graph
+// the fork and join become graph edges.)  The auxiliary stream and events
+// are created once per device on the first call made outside stream capture;
+// until then, and whenever the prefix grid would take more than half the
+// SMs, the two passes run one after the other on the caller's stream.
+namespace {
+
+struct AuxStream {
+  cudaStream_t stream = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+};
+AuxStream g_aux[kMaxDevicesHost];
+
+const AuxStream* aux_stream(cudaStream_t s) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevicesHost) return nullptr;
+  AuxStream& a = g_aux[dev];
+  if (a.join != nullptr) return &a;
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(s, &cs) != cudaSuccess || cs != cudaStreamCaptureStatusNone) return nullptr;
+  if (a.stream == nullptr && cudaStreamCreateWithFlags(&a.stream, cudaStreamNonBlocking) != cudaSuccess) {
+    a.stream = nullptr;
+    return nullptr;
+  }
+  if (a.fork == nullptr && cudaEventCreateWithFlags(&a.fork, cudaEventDisableTiming) != cudaSuccess) {
+    a.fork = nullptr;
+    return nullptr;
+  }
+  if (cudaEventCreateWithFlags(&a.join, cudaEventDisableTiming) != cudaSuccess) {
+    a.join = nullptr;
+    return nullptr;
+  }
+  return &a;
+}
+
+constexpr double kPrefixShare = 0.43;  // share of the SMs the side-by-side prefix pass gets
+
+}  // namespace
+
 cudaError_t launch_decode_cascade(const PoolView& pool, const TableView& t, const void* q,
                                   int32_t num_q_heads, const int32_t* table_idx,
                                   const int32_t* seq_lens, int32_t batch,
@@ -109,22 +153,56 @@ cudaError_t launch_decode_cascade(const PoolView& pool, const TableView& t, cons
                                   int32_t num_groups, int64_t max_prefix_len, float scale, void* out,
                                   void* workspace, int32_t* err, cudaStream_t s) {
   if (batch == 0) return cudaSuccess;
-  const int grid = decode_grid_size();
-  const CascadeLayout L = cascade_layout(batch, num_q_heads, max_prefix_len, grid);
+  const int sms = decode_grid_size();
+  const CascadeLayout L = cascade_layout(batch, num_q_heads, max_prefix_len, sms);
   uint8_t* w = static_cast<uint8_t*>(workspace);
   int32_t* kv_start = reinterpret_cast<int32_t*>(w + L.start_off);
   float2* pre_ml = reinterpret_cast<float2*>(w + L.ml_off);
   float* pre_o = reinterpret_cast<float*>(w + L.o_off);
-  const int64_t capacity = static_cast<int64_t>(L.nsplit) * L.split_keys;
+  // Prefix-pass CTAs per key split: KV heads x query blocks (two 128-row Q
+  // tiles of 128 / G tokens) x groups.
+  const int G = num_q_heads / pool.num_kv_heads;
+  const int64_t per_split = static_cast<int64_t>(pool.num_kv_heads) * ((batch + 2 * (128 / G) - 1) / (2 * (128 / G))) *
+                            num_groups;
+  int32_t nsplit = L.nsplit, split_keys = L.split_keys;
+  const AuxStream* aux = nullptr;
+  if (L.nsplit > 0 && per_split > 0 && per_split <= kPrefixShare * sms) {
+    int64_t ns = std::llround(kPrefixShare * sms / static_cast<double>(per_split));
+    ns = std::max<int64_t>(1, std::min<int64_t>(ns, L.nsplit));
+    if (per_split * ns <= sms / 2) {
+      aux = aux_stream(s);
+      if (aux != nullptr) {
+        nsplit = static_cast<int32_t>(ns);
+        const int64_t per = (max_prefix_len + nsplit - 1) / nsplit;
+        split_keys = static_cast<int32_t>((per + 63) / 64 * 64);
+      }
+    }
+  }
+  const int64_t capacity = static_cast<int64_t>(nsplit) * split_keys;
   cudaError_t e = launch_cascade_prep(group_offsets, group_prefix, num_groups, seq_lens, batch, capacity,
                                       kv_start, err, s);
   if (e != cudaSuccess) return e;
-  e = launch_extend_prefix(pool, t, q, num_q_heads, table_idx, group_offsets, group_prefix, num_groups, batch,
-                           L.nsplit, L.split_keys, scale, pre_ml, pre_o, err, s);
+  if (aux == nullptr) {
+    e = launch_extend_prefix(pool, t, q, num_q_heads, table_idx, group_offsets, group_prefix, num_groups, batch,
+                             nsplit, split_keys, scale, pre_ml, pre_o, err, s);
+    if (e != cudaSuccess) return e;
+    CascadeView cv{kv_start, pre_ml, pre_o, nsplit, nullptr};
+    return launch_decode(pool, t, q, num_q_heads, table_idx, seq_lens, batch, scale, out, w + L.decode_off, sms,
+                         err, s, &cv);
+  }
+  // Side by side: fork the auxiliary stream after the prep kernel, run the
+  // prefix pass there and the suffix pass here on the SMs it leaves free.
+  e = cudaEventRecord(aux->fork, s);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(aux->stream, aux->fork, 0);
   if (e != cudaSuccess) return e;
-  CascadeView cv{kv_start, pre_ml, pre_o, L.nsplit};
-  return launch_decode(pool, t, q, num_q_heads, table_idx, seq_lens, batch, scale, out, w + L.decode_off, grid,
-                       err, s, &cv);
+  e = launch_extend_prefix(pool, t, q, num_q_heads, table_idx, group_offsets, group_prefix, num_groups, batch,
+                           nsplit, split_keys, scale, pre_ml, pre_o, err, aux->stream);
+  if (e == cudaSuccess) e = cudaEventRecord(aux->join, aux->stream);
+  if (e != cudaSuccess) return e;
+  const int suffix_grid = static_cast<int>(sms - per_split * nsplit);
+  CascadeView cv{kv_start, pre_ml, pre_o, nsplit, aux->join};
+  return launch_decode(pool, t, q, num_q_heads, table_idx, seq_lens, batch, scale, out, w + L.decode_off,
+                       suffix_grid, err, s, &cv);
 }
 
 }  // namespace pkv

@@ -1453,6 +1453,10 @@ cudaError_t launch_split_t(const DecodeArgs& a, int grid, cudaStream_t s, const 
   cfg.numAttrs = 1;
   e = cudaLaunchKernelEx(&cfg, decode_split_kernel<E, G, kPaged>, a, kmap, vmap);
   if (e != cudaSuccess) return e;
+  if (cv != nullptr && cv->prefix_done != nullptr) {
+    e = cudaStreamWaitEvent(s, cv->prefix_done, 0);
+    if (e != cudaSuccess) return e;
+  }
   cudaLaunchConfig_t ccfg = cfg;
   ccfg.gridDim = dim3(a.batch, (a.hq + 3) / 4);
   ccfg.blockDim = dim3(128);

@@ -79,6 +79,9 @@ struct CascadeView {
   const float2* pre_ml;
   const float* pre_o;
   int32_t nsplit;
+  // When set, the prefix pass runs on another stream: the merge kernel's
+  // stream waits for this event (recorded after the prefix pass) first.
+  cudaEvent_t prefix_done = nullptr;
 };
 
 cudaError_t launch_decode(const PoolView& pool, const TableView& t, const void* q,
