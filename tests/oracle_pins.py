@@ -296,6 +296,20 @@ def pin_constant_k_mean_v(orc):
         _close(out[0, h], V[:, h // 2].mean(axis=0), 1e-14)
 
 
+def pin_constant_k_mean_v_group_16(orc):
+    """The same closed form at a GQA group of 16 (32 query heads over 2 KV
+    heads): query head h averages KV head h // 16's values."""
+    rng = np.random.default_rng(38)
+    n, Hkv, Hq = 13, 2, 32
+    k_row = _bf16_round(rng.standard_normal((Hkv, D)))
+    K = np.repeat(k_row[None], n, axis=0)
+    V = _bf16_round(rng.standard_normal((n, Hkv, D)))
+    q = _bf16_round(rng.standard_normal((1, Hq, D)))
+    out = orc.attend(_bits(q), _bits(K), _bits(V), [n], 0.5)
+    for h in range(Hq):
+        _close(out[0, h], V[:, h // 16].mean(axis=0), 1e-14)
+
+
 def pin_decode_equals_extend_one_row(orc):
     """decode over n tokens equals extend with prefix n-1 and one new row."""
     rng = np.random.default_rng(41)
@@ -355,7 +369,8 @@ def pin_empty_context_zero(orc):
 ALL_PINS = [pin_store_bit_copy, pin_page_translation_golden, pin_gather_matches_dense,
             pin_two_key_closed_form, pin_decode_brute_force, pin_extend_brute_force,
             pin_slot_permutation, pin_chunked_equals_unchunked, pin_shared_prefix_equals_private,
-            pin_one_token_returns_v, pin_constant_k_mean_v, pin_decode_equals_extend_one_row,
+            pin_one_token_returns_v, pin_constant_k_mean_v, pin_constant_k_mean_v_group_16,
+            pin_decode_equals_extend_one_row,
             pin_scale_invariance, pin_identical_heads, pin_split_combine, pin_empty_context_zero]
 
 
