@@ -26,6 +26,7 @@
 
 #include <algorithm>
 #include <cmath>
+#include <mutex>
 
 #include "common.cuh"
 #include "launch.h"
@@ -117,13 +118,17 @@ namespace {
 struct AuxStream {
   cudaStream_t stream = nullptr;
   cudaEvent_t fork = nullptr, join = nullptr;
+  // Held from the fork record to the join wait, so that calls from several
+  // host threads cannot interleave their records of the shared events.
+  std::mutex mu;
 };
 AuxStream g_aux[kMaxDevicesHost];
 
-const AuxStream* aux_stream(cudaStream_t s) {
+AuxStream* aux_stream(cudaStream_t s) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevicesHost) return nullptr;
   AuxStream& a = g_aux[dev];
+  std::lock_guard<std::mutex> lock(a.mu);  // released before the caller locks it again
   if (a.join != nullptr) return &a;
   cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
   if (cudaStreamIsCapturing(s, &cs) != cudaSuccess || cs != cudaStreamCaptureStatusNone) return nullptr;
@@ -165,7 +170,7 @@ cudaError_t launch_decode_cascade(const PoolView& pool, const TableView& t, cons
   const int64_t per_split = static_cast<int64_t>(pool.num_kv_heads) * ((batch + 2 * (128 / G) - 1) / (2 * (128 / G))) *
                             num_groups;
   int32_t nsplit = L.nsplit, split_keys = L.split_keys;
-  const AuxStream* aux = nullptr;
+  AuxStream* aux = nullptr;
   if (L.nsplit > 0 && per_split > 0 && per_split <= kPrefixShare * sms) {
     int64_t ns = std::llround(kPrefixShare * sms / static_cast<double>(per_split));
     ns = std::max<int64_t>(1, std::min<int64_t>(ns, L.nsplit));
@@ -192,6 +197,7 @@ cudaError_t launch_decode_cascade(const PoolView& pool, const TableView& t, cons
   }
   // Side by side: fork the auxiliary stream after the prep kernel, run the
   // prefix pass there and the suffix pass here on the SMs it leaves free.
+  std::lock_guard<std::mutex> lock(aux->mu);
   e = cudaEventRecord(aux->fork, s);
   if (e == cudaSuccess) e = cudaStreamWaitEvent(aux->stream, aux->fork, 0);
   if (e != cudaSuccess) return e;
