@@ -158,3 +158,51 @@ def test_cascade_host_checks():
     with pytest.raises(RuntimeError, match="invalid"):
         api.decode_attn_cascade(dd.pool, 0, dd.q, dd.table, dd.table_idx, dd.seq_lens, off,
                                 plen[:0], 64, out, ws, scale=wl.scale)
+
+
+def test_cascade_two_host_threads():
+    """Two host threads, each on its own stream, call the cascade at the same
+    time.  Each batch is one group of 256 requests, so both calls run the
+    prefix pass beside the suffix pass on the library's shared auxiliary
+    stream; every result must equal (bit for bit) the same call made alone."""
+    import threading
+    cases = []
+    for seed in (81, 82):
+        gd = W.grouped_decode(groups=((1000, 256),), max_suffix=150, seed=seed)
+        dd = DeviceDecode(gd.decode)
+        ref = _run_cascade(dd, gd.group_offsets, gd.group_prefix_lens).clone()
+        exp, _ = oracle_decode(gd.decode, requests=[0, 255])
+        tol_check(from_dev(ref)[[0, 255]], exp[[0, 255]], W.BF16, f"cascade seed {seed}")
+        cases.append((gd, dd, ref))
+    torch.cuda.synchronize()
+    failures = []
+
+    def worker(gd, dd, ref):
+        try:
+            st = torch.cuda.Stream()
+            wl = dd.wl
+            mp = int(np.max(gd.group_prefix_lens))
+            ws = api.decode_cascade_workspace(wl.batch, wl.num_q_heads, mp)
+            off, plen = i32(gd.group_offsets), i32(gd.group_prefix_lens)
+            torch.cuda.synchronize()
+            with torch.cuda.stream(st):
+                out = torch.empty_like(dd.q)
+                for _ in range(20):
+                    out.fill_(0)
+                    api.decode_attn_cascade(dd.pool, wl.layer, dd.q, dd.table, dd.table_idx, dd.seq_lens,
+                                            off, plen, mp, out, ws, scale=wl.scale, dev_err=dd.err)
+                    st.synchronize()
+                    if not torch.equal(out, ref):
+                        failures.append("a threaded call differs from the same call made alone")
+                        return
+        except Exception as exc:  # surfaced below
+            failures.append(repr(exc))
+
+    threads = [threading.Thread(target=worker, args=c) for c in cases]
+    for t in threads:
+        t.start()
+    for t in threads:
+        t.join(timeout=120)
+    assert not any(t.is_alive() for t in threads), "a worker thread did not finish"
+    assert not failures, failures[0]
+    assert all(int(c[1].err.item()) == 0 for c in cases)
