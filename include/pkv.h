@@ -356,6 +356,12 @@ int pkv_decode_attn_noalloc(const pkv_pool* pool, int32_t layer, const void* q,
  * once per request); each request's own suffix goes through the split-KV
  * decode kernel; the partial results are merged by their (max, sum) pairs.
  * This is not on the pages; it is the reuse their prefix sharing allows.
+ * When the prefix pass is small (about 43% of the SMs' worth of CTAs or
+ * less), it runs on a library-owned auxiliary stream beside the suffix pass,
+ * forked from and joined back to `stream` with events, so the call stays
+ * ordered on `stream` as a whole.  The auxiliary stream and its two events
+ * are created once per device, on the first call made outside stream
+ * capture; calls from several host threads are serialised around them.
  *
  * group_offsets: device int32 [num_groups + 1], 0 = first <= ... <= last =
  *   batch.  group_prefix_lens: device int32 [num_groups], each 0 <= p_g <=
@@ -366,7 +372,7 @@ int pkv_decode_attn_noalloc(const pkv_pool* pool, int32_t layer, const void* q,
  * workspace: pkv_decode_cascade_workspace_bytes(batch, num_q_heads,
  *   max_prefix_len) bytes, 16-byte aligned.
  * bf16 and FP8 pools (PKV_ERR_UNSUPPORTED for fp32); other limits as
- * decode_attn.
+ * decode_attn, with num_q_heads/num_kv_heads at most 8.
  */
 size_t pkv_decode_cascade_workspace_bytes(int32_t batch, int32_t num_q_heads,
                                           int64_t max_prefix_len);
