@@ -111,3 +111,21 @@ def test_rope_store_step_inputs():
     # cos^2 + sin^2 = 1 for every stored angle (float32 table).
     assert np.allclose(cs[:, :64] ** 2 + cs[:, 64:] ** 2, 1.0, atol=1e-6)
     assert np.array_equal(cs[0, :64], np.ones(64)) and np.array_equal(cs[0, 64:], np.zeros(64))
+
+
+def test_fp8_pool_variant_of_the_tiled_qwen3_8b_pool():
+    """The E4M3 copy of the Qwen3-8B batch keeps the tiled pool: a code block
+    of the same shape, tiled over the same slots; table and lengths unchanged;
+    no NaN code."""
+    base = W.decode_qwen3_8b(num_layers=2)
+    wl = W.with_fp8_pool(base)
+    assert isinstance(wl.k_planes, W.TiledPlane) and isinstance(wl.v_planes, W.TiledPlane)
+    for plane, src in ((wl.k_planes, base.k_planes), (wl.v_planes, base.v_planes)):
+        assert plane.block.dtype == np.uint8 and plane.block.shape == src.block.shape
+        assert plane.num_slots == src.num_slots and plane.num_layers == src.num_layers
+        assert not np.any((plane.block & 0x7F) == 0x7F)
+    assert wl.pool.dtype == W.F8 and wl.pool.page_size == 16
+    assert np.array_equal(wl.page_table, base.page_table) and np.array_equal(wl.seq_lens, base.seq_lens)
+    # A slot of layer 1 reads the block row (num_slots + slot) mod block rows.
+    nb = wl.k_planes.block.shape[0]
+    assert np.array_equal(wl.k_planes[1][np.array([5])][0], wl.k_planes.block[(wl.pool.num_slots + 5) % nb])
