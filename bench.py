@@ -912,6 +912,21 @@ def run_radix(args, world, rank, local):
                 other.append((a, b))
     torch.cuda.synchronize()
     other_ms = sorted(a.elapsed_time(b) for a, b in other)[len(other) // 2]
+
+    # Both decode forms as the decode workloads time their roofline: the L
+    # decode calls captured once in a graph and replayed back to back, so no
+    # events sit between the calls (outside the timed step).
+    def decode_all(use_cascade):
+        for l in range(L):
+            decode(l, use_cascade)
+
+    reps = max(3, args.steps)
+    graph_ms = {}
+    for form in (True, False):
+        g = capture(torch, dev, lambda: decode_all(form), 2)
+        t = time_replays(torch, s, g, lambda: decode_all(form), reps) / (reps * L)
+        graph_ms[form] = (t, g is not None)
+        del g
     flops_layer = extend_flops(ext.num_q_heads, ext.causal_pairs())
     ext_flops = flops_layer * L * args.steps
     logical = decode_bytes(dec) * L * args.steps
@@ -945,6 +960,13 @@ def run_radix(args, world, rank, local):
                    "prefix_flops_per_layer": 4 * 128 * dec.num_q_heads * dec.batch * 4096,
                    "other_call": "decode_attn" if cascade else "decode_attn_cascade",
                    "other_ms_per_layer": round(other_ms, 4),
+                   "graph_ms_per_layer": round(graph_ms[cascade][0], 4),
+                   "other_graph_ms_per_layer": round(graph_ms[not cascade][0], 4),
+                   "timing": ("ms_per_layer: events around each call inside the timed step; "
+                              "other_ms_per_layer: the median of 6 such calls after it; *graph_ms_per_layer: "
+                              f"{reps} back-to-back replays of a graph of the {L} decode calls"
+                              + ("" if graph_ms[True][1] and graph_ms[False][1] else
+                                 " (capture failed: eager calls)")),
                    "note": "logical bytes count the shared 4096-token prefix once per request"},
         "store_kv": {"tokens": ext.total_q, "bytes_per_call": st_call,
                      "us_per_call": round(st_ms / (L * args.steps) * 1e3, 2), "gbs": round(st_gbs, 1),
