@@ -30,6 +30,23 @@ MUTATIONS = {
     "decode_drops_new_token": ("attend(q[r:r + 1], K, V, [n], scale)", "attend(q[r:r + 1], K, V, [n - 1], scale)"),
     "combine_forgets_l": ("den = (w * ls).sum(axis=0)", "den = w.sum(axis=0)"),
     "partial_max_wrong": ("p = np.exp(s - m[h])", "p = np.exp(s)"),
+    "decode_ignores_table_idx": (
+        "s = slots_of(page_table, int(table_idx[r]), n, page_size)\n        K = k_planes[layer][s]\n"
+        "        V = v_planes[layer][s]\n        out[r:r + 1]",
+        "s = slots_of(page_table, r, n, page_size)\n        K = k_planes[layer][s]\n"
+        "        V = v_planes[layer][s]\n        out[r:r + 1]"),
+    "extend_ignores_table_idx": (
+        "s = slots_of(page_table, int(table_idx[r]), n, page_size)\n        K = k_planes[layer][s]\n"
+        "        V = v_planes[layer][s]\n        out[base + idx]",
+        "s = slots_of(page_table, r, n, page_size)\n        K = k_planes[layer][s]\n"
+        "        V = v_planes[layer][s]\n        out[base + idx]"),
+    "extend_ignores_q_offsets": ("base = int(q_offsets[r])", "base = 0"),
+    "extend_drops_prefix": ("n = p + e\n", "n = e\n"),
+    "mask_includes_limit": ("allowed = np.arange(n)[None, :] < lim[:, None]",
+                            "allowed = np.arange(n)[None, :] <= lim[:, None]"),
+    "gather_returns_k_for_v": ("np.asarray(v_planes[layer][s])))", "np.asarray(k_planes[layer][s])))"),
+    "gather_ignores_table_idx": ("s = slots_of(page_table, int(table_idx[r]), int(seq_lens[r]), page_size)",
+                                 "s = slots_of(page_table, r, int(seq_lens[r]), page_size)"),
 }
 
 # The same for the q/k norm + RoPE oracle.
