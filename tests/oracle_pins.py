@@ -548,5 +548,24 @@ def pin_fp8_one_token_returns_dequantised_v(orc):
         assert np.array_equal(out[0, h], v_vals[0].reshape(Hkv, D)[h // 2])
 
 
+def pin_fp8_quantize_inverse_in_float32(orc):
+    """The inverse scale is a float32 quotient, worked by hand for s = 7 and
+    x = 91/1024 (bf16 0x3DB6):
+
+    * 2^26 / 7 = 9586980.57..., so RN32(1/7) = 9586981 * 2^-26, and
+      7 * 9586981 = 2^26 + 3: RN32(1/7) = (1 + 3 * 2^-26) / 7.
+    * x * RN32(1/7) = 13 * 2^-10 + 39 * 2^-36.  On [2^-7, 2^-6) a float32 step
+      is 2^-30 and 39 * 2^-36 is 0.61 of it, so the float32 product is
+      t = 13 * 2^-10 + 2^-30.
+    * E4M3's subnormal quantum is 2^-9: 13 * 2^-10 is 6.5 quanta, a tie, and t
+      lies above it, so t rounds to 7 quanta: code 0x07 (0x87 for -x).  With
+      the exact 1/7 the product would be the tie itself, which goes to the even
+      code 0x06."""
+    x = np.array([0x3DB6, 0xBDB6], dtype=np.uint16)
+    assert float(orc.to_f64(x[:1])[0]) == 91 / 1024
+    assert [int(c) for c in orc.quantize(x, 7.0)] == [0x07, 0x87]
+    assert [int(c) for c in orc.quantize(np.array([91 / 1024], dtype=np.float32), 7.0)] == [0x07]
+
+
 ALL_PINS += [pin_e4m3_codes, pin_e4m3_decode_table, pin_fp8_quantize_scale,
-             pin_fp8_one_token_returns_dequantised_v]
+             pin_fp8_one_token_returns_dequantised_v, pin_fp8_quantize_inverse_in_float32]

@@ -84,6 +84,30 @@ def test_fp8_store_saturates():
     assert np.any((rows & 0x7F) == 0x7E)  # some values did saturate
 
 
+def test_fp8_store_inverse_scale_is_a_float32_quotient():
+    """Scale 7: x = 91/1024 (bf16 0x3DB6) times the float32 1/7 lands one
+    float32 step above the E4M3 tie 6.5 * 2^-9 and stores code 0x07 (0x87 for
+    -x); the exact quotient would tie to the even code 0x06.  Both sides must
+    take the float32 path, in every slot of the rows."""
+    wl = W.with_fp8_pool(W.decode_small(), k_scale=7.0, v_scale=7.0)
+    k_new = wl.k_new.copy()
+    v_new = wl.v_new.copy()
+    k_new[:, 0::2] = 0x3DB6
+    v_new[:, 1::2] = 0xBDB6
+    wl.k_new, wl.v_new = k_new, v_new
+    d = DeviceDecode(wl)
+    api.store_kv(d.pool, 0, d.k_new, d.v_new, d.out_loc, d.err)
+    torch.cuda.synchronize()
+    assert int(d.err.item()) == 0
+    kp, vp = _oracle_store(wl)
+    got_k, got_v = _codes(d.pool.k[0]), _codes(d.pool.v[0])
+    assert np.array_equal(got_k, kp[0]) and np.array_equal(got_v, vp[0])
+    Hkv = wl.pool.num_kv_heads
+    rows_k = got_k[wl.out_loc].reshape(wl.batch, Hkv * D)
+    rows_v = got_v[wl.out_loc].reshape(wl.batch, Hkv * D)
+    assert np.all(rows_k[:, 0::2] == 0x07) and np.all(rows_v[:, 1::2] == 0x87)
+
+
 def test_fp8_gather_bit_exact():
     wl = W.with_fp8_pool(W.decode_paged_small(), seed=3)
     d = DeviceDecode(wl)

@@ -59,6 +59,17 @@ ROPE_MUTATIONS = {
     "v_gets_rotated": ("vl[loc[i]] = to_storage(v[i], storage)", "vl[loc[i]] = to_storage(k[i], storage)"),
     "k_not_normed": ("k = rope_rotate_half(rms_norm(k, k_norm_w, eps), positions, cos_sin_cache)",
                      "k = rope_rotate_half(k, positions, cos_sin_cache)"),
+    "q_not_normed": ("q = rope_rotate_half(rms_norm(q, q_norm_w, eps), positions, cos_sin_cache)",
+                     "q = rope_rotate_half(q, positions, cos_sin_cache)"),
+    "rope_cos_sin_swapped": ("cos = cs[:, None, :half]\n    sin = cs[:, None, half:]",
+                             "cos = cs[:, None, half:]\n    sin = cs[:, None, :half]"),
+    "rope_first_half_sign": ("x1 * cos - x2 * sin", "x1 * cos + x2 * sin"),
+    "norm_weight_dropped": ("return x / np.sqrt(ms + eps) * w", "return x / np.sqrt(ms + eps)"),
+    "k_v_slices_swapped": ("k = qkv[:, Hq * d:(Hq + Hkv) * d].reshape(N, Hkv, d)\n"
+                           "    v = qkv[:, (Hq + Hkv) * d:].reshape(N, Hkv, d)",
+                           "v = qkv[:, Hq * d:(Hq + Hkv) * d].reshape(N, Hkv, d)\n"
+                           "    k = qkv[:, (Hq + Hkv) * d:].reshape(N, Hkv, d)"),
+    "bf16_keeps_7_bits": ("y = np.ldexp(np.rint(m * 256.0), e - 8)", "y = np.ldexp(np.rint(m * 128.0), e - 7)"),
 }
 
 
@@ -70,6 +81,13 @@ FP8_MUTATIONS = {
     "e4m3_subnormal_quantum": ("e = np.maximum(ex - 1, -6)", "e = np.maximum(ex - 1, -7)"),
     "quantize_divides": ("t = (xf * inv).astype(np.float32)", "t = (xf / inv).astype(np.float32)"),
     "dequant_forgets_scale": ("e4m3_decode(planes[l]) * float(np.float32(scale))", "e4m3_decode(planes[l])"),
+    "e4m3_sign_dropped": ("code = code | np.where(np.signbit(t), 0x80, 0)", "code = code"),
+    "e4m3_nan_codes_finite": ("v = np.where((c & 0x7F) == 0x7F, np.nan, v)", "v = v"),
+    "e4m3_subnormals_as_normals": ("v = np.where(e == 0, sub, normal)", "v = normal"),
+    "quantize_inverse_in_float64": ("inv = np.float32(1.0) / np.float32(scale)",
+                                    "inv = np.float64(1.0) / np.float64(scale)"),
+    "fp8_store_v_with_k_scale": ("vr = quantize(np.asarray(v_rows), v_scale)",
+                                 "vr = quantize(np.asarray(v_rows), k_scale)"),
 }
 
 
